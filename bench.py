@@ -1,0 +1,574 @@
+#!/usr/bin/env python
+"""Benchmark: effective TFLOP/s of the block-sparse attention forward on B200.
+
+Default workload: SD3-1024-like MMDiT joint attention (B=2 CFG pair, H=24,
+d=64, N = 256 text + 64x64 image tokens, block 64) with a seeded per-head mode
+table: 10 full heads, 11 arrow heads (window 1/2/4 blocks), 3 skip heads
+reusing a cached fp32 output. One step = the whole hot path on one batch:
+bsa_build_mask (arrow) + bsa_forward.
+
+Effective FLOPs count only computed blocks: 4 * block_q * block_k * d per kept
+(b, h, query block, KV block); skip heads count 0.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2|c1|c3|c4|c5s|c5f]
+  python bench.py --impl reference ...   (the fp64 oracle on host cores)
+Under torchrun every rank runs its own independent instance (weak scaling, no
+data-path collective); the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "effective TFLOP/s of block-sparse attn fwd & % of BF16 peak; speedup vs dense"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="bsa", choices=["bsa", "reference"])
+    ap.add_argument("--config", default="c2", choices=["c1", "c2", "c3", "c4", "c5s", "c5f"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, local_rank: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self.err = None
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = local_rank
+            if vis:
+                ids = [x.strip() for x in vis.split(",") if x.strip()]
+                if local_rank < len(ids) and ids[local_rank].isdigit():
+                    idx = int(ids[local_rank])
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # noqa: BLE001
+            self.err = repr(e)
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = get_r(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:  # noqa: BLE001
+                self.err = repr(e)
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._thr is not None:
+            self._thr.join()
+
+    def summary(self):
+        if self.nv is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": self.err}
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons - {"gpu_idle"}),
+               "samples": len(self.samples)}
+        if self.err:
+            out["error"] = self.err
+        return out
+
+
+# ----------------------------------------------------------------------------- jobs
+
+def _bsa():
+    import block_sparse_attention_37_b200 as bsa
+    bsa.library()
+    return bsa
+
+
+def source_sha():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "block_sparse_attention_37_b200", "csrc")
+    for f in ("attention.cu", "attention.cuh", "common.cuh"):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(key):
+    """DRAM bytes per launch from the committed ncu summary, if it matches today's kernel."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(key)
+    if not e or e.get("source_sha") != source_sha():
+        return None
+    return e.get("bytes_per_launch")
+
+
+class Job:
+    """One hot-path instance on one GPU. Subclasses fill in the step."""
+    name = ""
+    launches_per_step = 0
+
+    def step(self, ev_fwd=None):  # ev_fwd: (start, end) events around the forward launch
+        raise NotImplementedError
+
+
+class ArrowJob(Job):
+    """MMDiT joint attention with per-head full / arrow / skip modes."""
+
+    def __init__(self, w, dense=False):
+        bsa = _bsa()
+        self.bsa = bsa
+        s = w["shape"]
+        self.s = s
+        self.dm = bsa.dims(s.B, s.H, s.N, s.d, s.block_q, s.block_k, s.n_text)
+        self.host = {"q": w["q"], "k": w["k"], "v": w["v"],
+                     "modes": torch.from_numpy(np.zeros_like(w["head_mode"]) if dense else w["head_mode"]),
+                     "wins": torch.from_numpy(w["window"]),
+                     "cache": w.get("cache")}
+        dev = {k: (v.cuda() if v is not None else None) for k, v in self.host.items()}
+        self.q, self.k, self.v = dev["q"], dev["k"], dev["v"]
+        self.modes, self.wins, self.cache = dev["modes"], dev["wins"], dev["cache"]
+        self.blocks = bsa.BlockList.empty(s.B, s.H, s.n_qb, s.n_kb, bitmap=False)
+        self.o = torch.empty_like(self.q)
+        self.launches_per_step = 2
+        self.step()
+        torch.cuda.synchronize()
+        cnt = self.blocks.cnt.to(torch.int64)
+        self.blocks_computed = int(cnt.sum())
+        self.blocks_total = s.B * s.H * s.n_qb * s.n_kb
+        self.flops = 4.0 * s.block_q * s.block_k * s.d * self.blocks_computed
+
+    def step(self, ev_fwd=None):
+        bsa = self.bsa
+        bsa.build_mask(self.dm, bsa.MASK_ARROW, self.blocks, head_mode=self.modes, window=self.wins)
+        if ev_fwd:
+            ev_fwd[0].record()
+        bsa.forward(self.dm, self.q, self.k, self.v, self.o, self.modes, blocks=self.blocks, cache_in=self.cache)
+        if ev_fwd:
+            ev_fwd[1].record()
+
+    def e2e_setup(self):
+        self.pin = {k: (v.pin_memory() if v is not None else None) for k, v in self.host.items()}
+        self.o_host = torch.empty(self.o.shape, dtype=self.o.dtype).pin_memory()
+        self.h2d = sum(v.numel() * v.element_size() for v in self.pin.values() if v is not None)
+        self.d2h = self.o_host.numel() * self.o_host.element_size()
+
+    def e2e_step(self):
+        for name, dst in (("q", self.q), ("k", self.k), ("v", self.v), ("modes", self.modes),
+                          ("wins", self.wins), ("cache", self.cache)):
+            if self.pin[name] is not None:
+                dst.copy_(self.pin[name], non_blocking=True)
+        self.step()
+        self.o_host.copy_(self.o, non_blocking=True)
+
+
+class ContentJob(Job):
+    """FLUX-2048-like pooled top-k selection followed by the sparse forward."""
+
+    def __init__(self, w, dense=False):
+        bsa = _bsa()
+        self.bsa = bsa
+        s = w["shape"]
+        self.s = s
+        self.dm = bsa.dims(s.B, s.H, s.N, s.d, s.block_q, s.block_k, s.n_text)
+        self.q, self.k, self.v = (t.cuda() for t in (w["q"], w["k"], w["v"]))
+        self.modes = torch.full((s.H,), 0 if dense else 1, dtype=torch.int32, device="cuda")
+        self.spec = bsa.select_spec(bsa.SELECT_POOLED_QK, w["groups"], True)
+        self.ws = torch.empty(bsa.select_workspace_size(self.dm, self.spec), dtype=torch.uint8, device="cuda")
+        self.blocks = bsa.BlockList.empty(s.B, s.H, s.n_qb, s.n_kb, bitmap=False)
+        self.o = torch.empty_like(self.q)
+        self.dense = dense
+        self.launches_per_step = 3
+        self.step()
+        torch.cuda.synchronize()
+        self.blocks_total = s.B * s.H * s.n_qb * s.n_kb
+        self.blocks_computed = self.blocks_total if dense else int(self.blocks.cnt.to(torch.int64).sum())
+        self.flops = 4.0 * s.block_q * s.block_k * s.d * self.blocks_computed
+
+    def step(self, ev_fwd=None):
+        bsa = self.bsa
+        bsa.select_topk(self.dm, self.q, self.k, self.spec, self.blocks, self.ws)
+        if ev_fwd:
+            ev_fwd[0].record()
+        bsa.forward(self.dm, self.q, self.k, self.v, self.o, self.modes, blocks=self.blocks)
+        if ev_fwd:
+            ev_fwd[1].record()
+
+
+class DlmJob(Job):
+    """SparseD-like: one full-score selection at setup, then forwards reusing the mask."""
+
+    def __init__(self, w, dense=False, n_sets=2):
+        bsa = _bsa()
+        self.bsa = bsa
+        s = w["shape"]
+        self.s = s
+        self.dm = bsa.dims(s.B, s.H, s.N, s.d, s.block_q, s.block_k, s.n_text)
+        self.bias = w["bias"].cuda()
+        self.sets = [tuple(t.cuda() for t in W.dlm_step_qkv(s, 3, t)) for t in range(n_sets)]
+        self.modes = torch.full((s.H,), 0 if dense else 1, dtype=torch.int32, device="cuda")
+        spec = bsa.select_spec(bsa.SELECT_FULL_SCORE, w["groups"], False, s.d ** -0.5)
+        ws = torch.empty(bsa.select_workspace_size(self.dm, spec), dtype=torch.uint8, device="cuda")
+        self.blocks = bsa.BlockList.empty(s.B, s.H, s.n_qb, s.n_kb, bitmap=False)
+        q0, k0, _ = self.sets[0]
+        bsa.select_topk(self.dm, q0, k0, spec, self.blocks, ws, bias=self.bias)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        bsa.select_topk(self.dm, q0, k0, spec, self.blocks, ws, bias=self.bias)
+        e1.record()
+        torch.cuda.synchronize()
+        self.selection_ms = e0.elapsed_time(e1)
+        self.o = torch.empty_like(q0)
+        self.i = 0
+        self.launches_per_step = 1
+        self.blocks_total = s.B * s.H * s.n_qb * s.n_kb
+        self.blocks_computed = self.blocks_total if dense else int(self.blocks.cnt.to(torch.int64).sum())
+        self.flops = 4.0 * s.block_q * s.block_k * s.d * self.blocks_computed
+
+    def step(self, ev_fwd=None):
+        q, k, v = self.sets[self.i % len(self.sets)]
+        self.i += 1
+        if ev_fwd:
+            ev_fwd[0].record()
+        self.bsa.forward(self.dm, q, k, v, self.o, self.modes, blocks=self.blocks, bias=self.bias)
+        if ev_fwd:
+            ev_fwd[1].record()
+
+
+class VideoJob(Job):
+    """GNA-like 3-D neighborhood attention: permute, mask, forward, unpermute."""
+
+    def __init__(self, w, dense=False):
+        bsa = _bsa()
+        self.bsa = bsa
+        s = w["shape"]
+        g = w["geom"]
+        self.geom = bsa.GnaGeom.make(g.grid, g.tile, g.window, g.stride)
+        nt = bsa.gna_tiled_len(s.n_text, self.geom)
+        self.dm_r = bsa.dims(s.B, s.H, s.N, s.d, s.block_q, s.block_k, s.n_text)
+        self.dm = bsa.dims(s.B, s.H, nt, s.d, s.block_q, s.block_k, s.n_text)
+        self.raster = [t.cuda() for t in (w["q"], w["k"], w["v"])]
+        self.tiled = [torch.empty((s.B, s.H, nt, s.d), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+        self.modes = torch.full((s.H,), 0 if dense else 1, dtype=torch.int32, device="cuda")
+        nb = nt // s.block_q
+        self.blocks = bsa.BlockList.empty(s.B, s.H, nb, nb, bitmap=False)
+        self.o_t = torch.empty_like(self.tiled[0])
+        self.o = torch.empty_like(self.raster[0])
+        self.launches_per_step = 4
+        self.step()
+        torch.cuda.synchronize()
+        self.blocks_total = s.B * s.H * nb * nb
+        self.blocks_computed = int(self.blocks.cnt.to(torch.int64).sum())
+        self.flops = 4.0 * s.block_q * s.block_k * s.d * self.blocks_computed
+
+    def step(self, ev_fwd=None):
+        bsa = self.bsa
+        bsa.permute_tiles(self.dm_r, self.geom, self.raster, self.tiled)
+        bsa.build_mask(self.dm, bsa.MASK_GNA, self.blocks, head_mode=self.modes, gna=self.geom)
+        if ev_fwd:
+            ev_fwd[0].record()
+        bsa.forward(self.dm, *self.tiled, self.o_t, self.modes, blocks=self.blocks, gna=self.geom)
+        if ev_fwd:
+            ev_fwd[1].record()
+        bsa.unpermute_tiles(self.dm_r, self.geom, [self.o_t], [self.o])
+
+
+CONFIGS = {
+    "c1": ("tiny arrow: B=1 H=2 d=64 N=512 (64 text + 16x28), block 64, head0 full, head1 arrow w=1",
+           lambda seed: W.c1(seed), ArrowJob),
+    "c2": ("SD3-1024-like MMDiT joint attention: B=2 H=24 d=64 N=4352 (256 text + 64x64), block 64, "
+           "modes 10 full / 11 arrow (w in {1,2,4}) / 3 skip (cached fp32 output)",
+           lambda seed: W.c2(seed), ArrowJob),
+    "c3": ("FLUX-2048-like pooled selection: B=1 H=24 d=128 N=16896 (512 text + 128x128), block 128, "
+           "top-30% image KV blocks + text", lambda seed: W.c3(seed), ContentJob),
+    "c4": ("SparseD-like DLM: B=1 H=32 d=128 N=32768 (30720 prefill + 2048 gen), block 128, "
+           "isolated top-30% full-score selection reused across steps", lambda seed: W.c4(seed), DlmJob),
+    "c5s": ("GNA-like video: B=1 H=24 d=128 256 text + 16x48x80, tile 4x8x8, window 8x16x24, stride 4x8x8",
+            lambda seed: W.c5((4, 8, 8), seed), VideoJob),
+    "c5f": ("GNA-like video: B=1 H=24 d=128 256 text + 16x48x80, tile 4x8x8, window 8x16x24, stride 1x1x1",
+            lambda seed: W.c5((1, 1, 1), seed), VideoJob),
+}
+DEFAULT_SEEDS = {"c1": 0, "c2": 1, "c3": 2, "c4": 3, "c5s": 4, "c5f": 4}
+
+
+# ----------------------------------------------------------------------------- timing
+
+def time_steps(job, steps, warmup, flush, with_fwd_events=True):
+    """Per-step device time (CUDA events on the launching stream), L2 flushed before each step."""
+    for _ in range(warmup):
+        flush.zero_()
+        job.step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e in evs:
+        flush.zero_()
+        e[0].record()
+        job.step((e[2], e[3]) if with_fwd_events else None)
+        e[1].record()
+    torch.cuda.synchronize()
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    fwd_ms = [e[2].elapsed_time(e[3]) for e in evs] if with_fwd_events else None
+    return step_ms, fwd_ms
+
+
+def oracle_sample_tflops(cfg, budget_s, seed=0):
+    """Time the fp64 oracle on a bounded sample of the workload (host cores)."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import attention as OA
+    from oracle import masks as OM
+    w = CONFIGS[cfg][1](DEFAULT_SEEDS[cfg])
+    if cfg not in ("c1", "c2"):
+        w = W.c2(1)  # the oracle baseline is taken on the arrow workload
+    s = w["shape"]
+    rng = np.random.default_rng(seed)
+    heads = [(b, h) for b in range(s.B) for h in range(s.H) if int(w["head_mode"][h]) != W.HEAD_SKIP]
+    order = [heads[i] for i in rng.permutation(len(heads))]
+    flops = 0.0
+    done = 0
+    t0 = time.perf_counter()
+    for (b, h) in order:
+        mode = int(w["head_mode"][h])
+        fn = lambda r, h=h, mode=mode: OM.arrow_token_mask(s.N, s.n_text, s.block_q, mode, int(w["window"][h]), r)
+        OA.head_forward(w["q"][b, h].double().numpy(), w["k"][b, h].double().numpy(),
+                        w["v"][b, h].double().numpy(), mode, fn, s.d ** -0.5)
+        nb = s.n_kb
+        if mode == W.HEAD_FULL:
+            kept = nb * nb
+        else:
+            kept = int((OM.arrow_block_classes(s.N, s.n_text, s.block_q, mode, int(w["window"][h])) > 0).sum())
+        flops += 4.0 * s.block_q * s.block_k * s.d * kept
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    el = time.perf_counter() - t0
+    threads = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas") or 1
+    return {"value": flops / el / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
+            "sample": f"{done} of {len(heads)} computed (b,h) heads of the SD3-1024-like workload, all rows, "
+                      f"{el:.1f} s wall", "seconds": el}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, rank, world):
+    """--impl reference: the oracle on host cores (rank 0 only)."""
+    if rank != 0:
+        return 0
+    cfg = args.config
+    desc = CONFIGS[cfg][0] if cfg in ("c1", "c2") else CONFIGS["c2"][0]
+    per_step = max(0.2, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        oracle_sample_tflops(cfg, per_step * 0.2)
+    vals, secs = [], []
+    res = None
+    for i in range(args.steps):
+        res = oracle_sample_tflops(cfg, per_step, seed=i)
+        vals.append(res["value"])
+        secs.append(res["seconds"])
+    value = float(np.median(vals))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * float(np.mean(secs)),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": desc, "impl": "fp64 numpy oracle on host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": res["cores"], "kind": "oracle",
+                         "sample": res["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_bsa(args, rank, world, local_rank):
+    import torch.distributed as dist
+    peaks, peak_src = load_peaks()
+    cfg = args.config
+    desc, make, JobT = CONFIGS[cfg]
+    seed = DEFAULT_SEEDS[cfg] + 1000 * rank
+    w = make(seed)
+    job = JobT(w)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+
+    sampler = ClockSampler(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    wall0 = time.perf_counter()
+    step_ms, fwd_ms = time_steps(job, args.steps, args.warmup, flush)
+    torch.cuda.synchronize()
+    wall1 = time.perf_counter()
+    sampler.stop()
+    if world > 1:
+        dist.barrier()
+    total_ms = float(np.sum(step_ms))
+    t = torch.tensor([total_ms, float(np.sum(fwd_ms))], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_total = float(t[0]), float(t[1])
+    ms_per_step = total_ms / args.steps
+    fwd_ms_mean = fwd_total / args.steps
+    value = job.flops * world / (ms_per_step * 1e-3) / 1e12
+
+    extra = {}
+    if not args.no_dense:
+        dense = JobT(w, dense=True)
+        d_step, d_fwd = time_steps(dense, max(10, args.steps // 4), args.warmup, flush)
+        sparsity = 1.0 - job.blocks_computed / job.blocks_total
+        extra = {"dense_fwd_ms": float(np.mean(d_fwd)), "fwd_ms": fwd_ms_mean,
+                 "speedup_vs_dense": float(np.mean(d_fwd)) / fwd_ms_mean,
+                 "ideal_speedup": 1.0 / (1.0 - sparsity) if sparsity < 1 else None,
+                 "block_sparsity": sparsity,
+                 "dense_tflops": dense.flops / (float(np.mean(d_fwd)) * 1e-3) / 1e12}
+        del dense
+    if isinstance(job, DlmJob):
+        extra["selection_ms"] = job.selection_ms
+
+    e2e = None
+    if not args.no_e2e and hasattr(job, "e2e_setup"):
+        job.e2e_setup()
+        for _ in range(max(3, args.warmup // 4)):
+            job.e2e_step()
+        torch.cuda.synchronize()
+        n = max(10, min(200, args.steps // 10))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            job.e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n
+        te = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": job.flops * world / (float(te[0]) * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": int(job.h2d), "d2h_bytes_per_step": int(job.d2h),
+               "ms_per_step": float(te[0])}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_sample_tflops(cfg, args.cpu_seconds)
+        cpu.pop("seconds", None)
+
+    peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    achieved = job.flops / (fwd_ms_mean * 1e-3) / 1e12
+    key = f"attn_fwd_{cfg}"
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": traffic_for(key),
+            "kernel": "bsa::attn_kernel<D,KIND_FWD> (bsa_forward)",
+            "peak_source": f"{peak_src} bf16 burst (kernel timed alone between L2 flushes)",
+            "algorithmic_flops_per_launch": job.flops}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the pages' workloads)",
+        "config": {"workload": desc, "config": cfg,
+                   "l2": "flushed before every step (256 MiB write), flush outside the timed events",
+                   "parallelism": f"independent replica per GPU x{world}", "seed": DEFAULT_SEEDS[cfg]},
+        "pct_of_bf16_peak": 100.0 * value / world / peak,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": job.launches_per_step * args.steps,
+        "clocks": sampler.summary(),
+        "wall_s_timed_region": wall1 - wall0,
+        "blocks_computed": job.blocks_computed, "blocks_total": job.blocks_total,
+    }
+    line.update(extra)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        return run_bsa(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

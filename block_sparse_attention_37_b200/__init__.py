@@ -1,0 +1,249 @@
+"""Python binding of libbsa.so (include/bsa.h): argument marshalling only.
+
+Every call here converts torch tensors to device pointers and forwards to the
+C ABI of the same name; all computation runs in the library's CUDA kernels.
+There is no CPU path: tensors must live on a CUDA device, and importing the
+binding without the built library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbsa.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(6)
+DEVERR_NONE, DEVERR_BAD_INDEX, DEVERR_TIMEOUT, DEVERR_SCHEDULE, DEVERR_NO_GEOMETRY = range(5)
+HEAD_FULL, HEAD_SPARSE, HEAD_SKIP = 0, 1, 2
+BLOCK_NONE, BLOCK_FULL, BLOCK_PARTIAL = 0, 1, 2
+MASK_ARROW, MASK_GNA = 1, 2
+SELECT_POOLED_QK, SELECT_FULL_SCORE = 1, 2
+
+EXPORTS = (
+    "bsa_version", "bsa_error_string", "bsa_build_mask", "bsa_select_workspace_size",
+    "bsa_select_topk", "bsa_forward", "bsa_gna_tiled_len", "bsa_permute_tiles",
+    "bsa_unpermute_tiles", "bsa_get_device_error",
+)
+
+
+class BsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_lib().bsa_error_string(status).decode()} (status {status})")
+
+
+# ---------------------------------------------------------------------------- structs
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("block_q", ctypes.c_int32), ("block_k", ctypes.c_int32),
+                ("n_text", ctypes.c_int32)]
+
+
+class GnaGeom(ctypes.Structure):
+    _fields_ = [("ndim", ctypes.c_int32), ("grid", ctypes.c_int32 * 3), ("tile", ctypes.c_int32 * 3),
+                ("window", ctypes.c_int32 * 3), ("stride", ctypes.c_int32 * 3)]
+
+    @classmethod
+    def make(cls, grid, tile, window, stride):
+        n = len(grid)
+        g = cls()
+        g.ndim = n
+        for i in range(n):
+            g.grid[i], g.tile[i], g.window[i], g.stride[i] = grid[i], tile[i], window[i], stride[i]
+        return g
+
+
+class MaskSpec(ctypes.Structure):
+    _fields_ = [("kind", ctypes.c_int32), ("head_mode", ctypes.c_void_p), ("window", ctypes.c_void_p),
+                ("gna", GnaGeom)]
+
+
+class BlockListC(ctypes.Structure):
+    _fields_ = [("cnt", ctypes.c_void_p), ("idx", ctypes.c_void_p), ("flag", ctypes.c_void_p),
+                ("bitmap", ctypes.c_void_p), ("max_k", ctypes.c_int32)]
+
+
+class KeyGroup(ctypes.Structure):
+    _fields_ = [("begin", ctypes.c_int32), ("end", ctypes.c_int32), ("k", ctypes.c_int32)]
+
+
+class SelectSpec(ctypes.Structure):
+    _fields_ = [("method", ctypes.c_int32), ("n_groups", ctypes.c_int32), ("groups", KeyGroup * 4),
+                ("keep_text", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+# ---------------------------------------------------------------------------- library
+
+_LIB = None
+
+
+def _lib():
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libbsa.so not built at {LIB_PATH}: run "
+                              "python -m block_sparse_attention_37_b200.build")
+        lib = ctypes.CDLL(LIB_PATH)
+        P = ctypes.c_void_p
+        lib.bsa_version.restype = ctypes.c_int
+        lib.bsa_error_string.restype = ctypes.c_char_p
+        lib.bsa_error_string.argtypes = [ctypes.c_int]
+        lib.bsa_build_mask.argtypes = [P, P, P, P]
+        lib.bsa_select_workspace_size.restype = ctypes.c_size_t
+        lib.bsa_select_workspace_size.argtypes = [P, P]
+        lib.bsa_select_topk.argtypes = [P, P, P, P, P, P, ctypes.c_size_t, P, P]
+        lib.bsa_forward.argtypes = [P, P, P, P, P, P, P, P, P, P, ctypes.c_float, P, P]
+        lib.bsa_gna_tiled_len.argtypes = [ctypes.c_int32, P, P]
+        lib.bsa_permute_tiles.argtypes = [P, P, ctypes.c_int32, P, P, P]
+        lib.bsa_unpermute_tiles.argtypes = [P, P, ctypes.c_int32, P, P, P]
+        lib.bsa_get_device_error.argtypes = [P, P]
+        _LIB = lib
+    return _LIB
+
+
+def library():
+    """The loaded ctypes library (raises ImportError if it was not built)."""
+    return _lib()
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise BsaError(status, where)
+
+
+def _ptr(t, dtype=None, name="tensor"):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device (the library has no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def version() -> int:
+    return _lib().bsa_version()
+
+
+def dims(B, H, N, d, block_q, block_k, n_text) -> Dims:
+    return Dims(B, H, N, d, block_q, block_k, n_text)
+
+
+def n_blocks(n: int, bs: int) -> int:
+    return -(-n // bs)
+
+
+@dataclass
+class BlockList:
+    """Device buffers of a block list (see bsa_block_list)."""
+    cnt: torch.Tensor
+    idx: torch.Tensor
+    flag: torch.Tensor
+    bitmap: torch.Tensor | None
+    max_k: int
+
+    @classmethod
+    def empty(cls, B, H, nQB, nKB, max_k=None, device="cuda", bitmap=True):
+        max_k = nKB if max_k is None else max_k
+        return cls(
+            cnt=torch.empty((B, H, nQB), dtype=torch.int32, device=device),
+            idx=torch.empty((B, H, nQB, max_k), dtype=torch.int32, device=device),
+            flag=torch.empty((B, H, nQB, max_k), dtype=torch.uint8, device=device),
+            bitmap=torch.empty((B, H, nQB, nKB), dtype=torch.uint8, device=device) if bitmap else None,
+            max_k=max_k)
+
+    def c(self) -> BlockListC:
+        return BlockListC(_ptr(self.cnt, torch.int32, "cnt"), _ptr(self.idx, torch.int32, "idx"),
+                          _ptr(self.flag, torch.uint8, "flag"),
+                          _ptr(self.bitmap, torch.uint8, "bitmap"), self.max_k)
+
+
+# ---------------------------------------------------------------------------- calls
+
+def build_mask(dm: Dims, kind: int, out: BlockList, head_mode=None, window=None, gna: GnaGeom | None = None,
+               stream=None):
+    spec = MaskSpec(kind, _ptr(head_mode, torch.int32, "head_mode"), _ptr(window, torch.int32, "window"),
+                    gna if gna is not None else GnaGeom())
+    lc = out.c()
+    _check(_lib().bsa_build_mask(ctypes.byref(dm), ctypes.byref(spec), ctypes.byref(lc), _stream(stream)),
+           "bsa_build_mask")
+
+
+def select_spec(method: int, groups, keep_text: bool, scale: float = 1.0) -> SelectSpec:
+    sp = SelectSpec()
+    sp.method = method
+    sp.n_groups = len(groups)
+    for i, (b, e, k) in enumerate(groups):
+        sp.groups[i] = KeyGroup(b, e, k)
+    sp.keep_text = 1 if keep_text else 0
+    sp.scale = scale
+    return sp
+
+
+def select_workspace_size(dm: Dims, spec: SelectSpec) -> int:
+    return int(_lib().bsa_select_workspace_size(ctypes.byref(dm), ctypes.byref(spec)))
+
+
+def select_topk(dm: Dims, q, k, spec: SelectSpec, out: BlockList, workspace, bias=None, stream=None):
+    lc = out.c()
+    _check(_lib().bsa_select_topk(ctypes.byref(dm), _ptr(q, torch.bfloat16, "Q"), _ptr(k, torch.bfloat16, "K"),
+                                  ctypes.byref(spec), _ptr(bias, torch.float32, "bias"),
+                                  _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+                                  ctypes.byref(lc), _stream(stream)), "bsa_select_topk")
+
+
+def forward(dm: Dims, q, k, v, o, head_mode, blocks: BlockList | None = None, gna: GnaGeom | None = None,
+            cache_in=None, cache_out=None, bias=None, scale: float | None = None, stream=None):
+    scale = (1.0 / dm.d ** 0.5) if scale is None else scale
+    lc = blocks.c() if blocks is not None else None
+    _check(_lib().bsa_forward(ctypes.byref(dm), _ptr(q, torch.bfloat16, "Q"), _ptr(k, torch.bfloat16, "K"),
+                              _ptr(v, torch.bfloat16, "V"), ctypes.byref(lc) if lc is not None else None,
+                              _ptr(head_mode, torch.int32, "head_mode"),
+                              ctypes.byref(gna) if gna is not None else None,
+                              _ptr(cache_in, torch.float32, "cache_in"), _ptr(cache_out, torch.float32, "cache_out"),
+                              _ptr(bias, torch.float32, "bias"), float(scale), _ptr(o, torch.bfloat16, "O"),
+                              _stream(stream)), "bsa_forward")
+
+
+def gna_tiled_len(n_text: int, gna: GnaGeom) -> int:
+    n = ctypes.c_int32(0)
+    _check(_lib().bsa_gna_tiled_len(int(n_text), ctypes.byref(gna), ctypes.byref(n)), "bsa_gna_tiled_len")
+    return int(n.value)
+
+
+def _ptr_array(ts, name):
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = _ptr(t, torch.bfloat16, f"{name}[{i}]").value
+    return arr
+
+
+def permute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
+    _check(_lib().bsa_permute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), _ptr_array(ins, "in"),
+                                    _ptr_array(outs, "out"), _stream(stream)), "bsa_permute_tiles")
+
+
+def unpermute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
+    _check(_lib().bsa_unpermute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), _ptr_array(ins, "in"),
+                                      _ptr_array(outs, "out"), _stream(stream)), "bsa_unpermute_tiles")
+
+
+def get_device_error(stream=None) -> int:
+    code = ctypes.c_int32(0)
+    _check(_lib().bsa_get_device_error(_stream(stream), ctypes.byref(code)), "bsa_get_device_error")
+    return int(code.value)

@@ -1,0 +1,38 @@
+// Parameters and launcher of the tcgen05 attention kernel (attention.cu).
+#pragma once
+
+#include "common.cuh"
+
+namespace bsa {
+
+enum { KIND_FWD = 0, KIND_LSE = 1, KIND_POOL = 2 };
+
+// 64-key segments per sequence the per-CTA schedule can hold: N <= 131072.
+constexpr int kMaxSeg = 2048;
+
+struct AttnParams {
+  int B, H, N;
+  int block_q, block_k, n_text;
+  int nQB, nKB, nQT, nSeg;
+  // block list (SPARSE heads)
+  const int32_t* cnt;
+  const int32_t* idx;
+  const uint8_t* flag;
+  int max_k;
+  const int32_t* head_mode;  // [H] (forward only)
+  const float* cache_in;     // [B,H,N,d] fp32, SKIP heads
+  float* cache_out;          // [B,H,N,d] fp32 or null
+  const float* bias;         // [H,nQB,nKB] fp32 or null (natural-log units)
+  float scale_log2;          // scale * log2(e)
+  __nv_bfloat16* O;          // [B,H,N,d]
+  float* lse;                // [B,H,N] log2-domain row LSE (LSE out, POOL in)
+  float* apool;              // [B,H,nQB,nKB] block sums of softmax (POOL out)
+  const int32_t* order;      // optional CTA -> work item permutation
+  int has_gna;
+  GnaDev g;
+};
+
+cudaError_t launch_attention(int d, int kind, const CUtensorMap& q, const CUtensorMap& k,
+                             const CUtensorMap& v, const AttnParams& p, int grid, cudaStream_t stream);
+
+}  // namespace bsa

@@ -1,0 +1,175 @@
+// Content-driven block selection.
+//  * block_pool_kernel: mean of every 64/128/256-token block of Q and K in
+//    fp32 (lmnt.cn BSA post, section 2.2, mean-pooled block vectors). HBM
+//    bound: 16-byte coalesced loads, eight blocks of loads in flight per CTA.
+//  * select_kernel: per (b, h, query block) row, the score of every KV block
+//    (pooled dot product, or the SparseD avg-pooled softmax mass from the
+//    attention kernel's POOL pass), then an exact rank-and-cut per key group
+//    (descending score, ties to the lower index) and an ascending block list.
+#include "select.cuh"
+
+namespace bsa {
+
+// grid: (nB, B*H, 2 tensors); block 256. out[t][bh][I][:] = mean of block I.
+template <int D>
+__global__ void __launch_bounds__(256) block_pool_kernel(PoolParams p) {
+  constexpr int CH = D / 8;           // 16-byte chunks per row
+  constexpr int RPI = 256 / CH;       // rows per iteration
+  __shared__ float red[RPI][D + 1];
+  const int I = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
+  const int bs = which ? p.block_k : p.block_q;
+  const int nb = which ? p.nKB : p.nQB;
+  if (I >= nb) return;
+  const __nv_bfloat16* src = (which ? p.K : p.Q) + ((size_t)bh * p.N) * D;
+  float* dst = (which ? p.kbar : p.qbar) + ((size_t)bh * nb + I) * D;
+  const int r0 = I * bs;
+  const int rows = min(bs, p.N - r0);
+  const int c = threadIdx.x % CH, rr = threadIdx.x / CH;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+  for (int base = 0; base < rows; base += RPI * 4) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int r = base + u * RPI + rr;
+      if (r < rows)
+        v[u] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)(r0 + r) * D) + c);
+      else
+        v[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(h2[j]);
+        acc[2 * j] += f.x;
+        acc[2 * j + 1] += f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[rr][c * 8 + j] = acc[j];
+  __syncthreads();
+  for (int col = threadIdx.x; col < D; col += 256) {
+    float s = 0.f;
+#pragma unroll 4
+    for (int q = 0; q < RPI; ++q) s += red[q][col];
+    dst[col] = s / (float)rows;
+  }
+}
+
+__device__ __forceinline__ float sanitize(float x) { return (x == x) ? x : -__int_as_float(0x7f800000); }
+
+// One CTA per (b, h, query block). Block 256 threads.
+template <int D>
+__global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
+  extern __shared__ float sc[];  // [nKB] scores
+  __shared__ float qv[D];
+  __shared__ int warp_tot[8];
+  uint8_t* keep = reinterpret_cast<uint8_t*>(sc + p.nKB);
+  const int I = blockIdx.x % p.nQB;
+  const int bh = blockIdx.x / p.nQB;
+  const size_t row = (size_t)bh * p.nQB + I;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (p.method == BSA_SELECT_POOLED_QK) {
+    for (int j = tid; j < D; j += 256) qv[j] = p.qbar[row * D + j];
+    __syncthreads();
+    const float* kb = p.kbar + (size_t)bh * p.nKB * D;
+    for (int J = tid; J < p.nKB; J += 256) {
+      const float4* kr = reinterpret_cast<const float4*>(kb + (size_t)J * D);
+      float s = 0.f;
+#pragma unroll 8
+      for (int j = 0; j < D / 4; ++j) {
+        const float4 k4 = __ldg(kr + j);
+        s = fmaf(qv[4 * j], k4.x, s);
+        s = fmaf(qv[4 * j + 1], k4.y, s);
+        s = fmaf(qv[4 * j + 2], k4.z, s);
+        s = fmaf(qv[4 * j + 3], k4.w, s);
+      }
+      sc[J] = sanitize(s);
+    }
+  } else {
+    const int nq = min(p.block_q, p.N - I * p.block_q);
+    for (int J = tid; J < p.nKB; J += 256) {
+      const int nk = min(p.block_k, p.N - J * p.block_k);
+      sc[J] = sanitize(p.apool[row * p.nKB + J] / ((float)nq * (float)nk));
+    }
+  }
+  for (int J = tid; J < p.nKB; J += 256) keep[J] = 0;
+  __syncthreads();
+
+  const bool full_row = p.keep_text && I < p.ntbq;
+  if (full_row) {
+    for (int J = tid; J < p.nKB; J += 256) keep[J] = 1;
+  } else {
+    if (p.keep_text)
+      for (int J = tid; J < min(p.ntbk, p.nKB); J += 256) keep[J] = 1;
+    for (int g = 0; g < p.n_groups; ++g) {
+      const int b = p.groups[g].begin, e = min(p.groups[g].end, p.nKB), k = p.groups[g].k;
+      for (int J = b + tid; J < e; J += 256) {
+        const float sj = sc[J];
+        int rank = 0;
+        for (int J2 = b; J2 < e; ++J2) {
+          const float s2 = sc[J2];
+          rank += (s2 > sj) || (s2 == sj && J2 < J);
+        }
+        if (rank < k) keep[J] = 1;
+      }
+    }
+  }
+  __syncthreads();
+
+  // ascending compaction
+  int32_t* idx = p.idx + row * p.max_k;
+  uint8_t* flag = p.flag + row * p.max_k;
+  int base = 0;
+  for (int J0 = 0; J0 < p.nKB; J0 += 256) {
+    const int J = J0 + tid;
+    const bool kk = J < p.nKB && keep[J];
+    const unsigned bal = __ballot_sync(0xffffffffu, kk);
+    if (lane == 0) warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < 8; ++w) {
+      before += (w < warp) ? warp_tot[w] : 0;
+      total += warp_tot[w];
+    }
+    if (kk) {
+      const int pos = base + before + __popc(bal & ((1u << lane) - 1u));
+      idx[pos] = J;
+      flag[pos] = BSA_BLOCK_FULL;
+    }
+    if (J < p.nKB && p.bitmap) p.bitmap[row * p.nKB + J] = kk ? BSA_BLOCK_FULL : BSA_BLOCK_NONE;
+    base += total;
+    __syncthreads();
+  }
+  for (int e = base + tid; e < p.max_k; e += 256) {
+    idx[e] = -1;
+    flag[e] = 0;
+  }
+  if (tid == 0) p.cnt[row] = base;
+}
+
+cudaError_t launch_block_pool(int d, const PoolParams& p, cudaStream_t stream) {
+  dim3 grid(max(p.nQB, p.nKB), p.B * p.H, 2);
+  if (d == 64)
+    block_pool_kernel<64><<<grid, 256, 0, stream>>>(p);
+  else
+    block_pool_kernel<128><<<grid, 256, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(int d, const SelectParams& p, cudaStream_t stream) {
+  const size_t smem = (size_t)p.nKB * sizeof(float) + (size_t)p.nKB;
+  const unsigned grid = (unsigned)((size_t)p.B * p.H * p.nQB);
+  if (d == 64)
+    select_kernel<64><<<grid, 256, smem, stream>>>(p);
+  else
+    select_kernel<128><<<grid, 256, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

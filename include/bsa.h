@@ -1,0 +1,206 @@
+/*
+ * bsa.h - block-sparse attention for diffusion transformers on B200 (sm_100a).
+ *
+ * A small C ABI over hand-written CUDA kernels. Every pointer argument named
+ * "device" is caller-owned device memory; the library never allocates, never
+ * synchronises the host (except bsa_get_device_error) and has no CPU fallback.
+ * All launches are asynchronous on the caller's stream, passed as `void*`
+ * holding a cudaStream_t (NULL = legacy default stream).
+ *
+ * Tensor layout: Q, K, V and O are bf16 [B, H, N, d], row-major, d innermost
+ * and contiguous, 16-byte aligned. Text tokens come first in the sequence,
+ * followed by the image (or video) tokens.
+ *
+ * Return values: BSA_OK or one of the BSA_ERR_* codes below. Argument checks
+ * happen on the host before any launch; a failed check launches nothing.
+ * Faults found by kernels (an out-of-range block index, a bounded pipeline
+ * wait that ran out) are recorded in a device error word, read with
+ * bsa_get_device_error.
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define BSA_OK 0
+#define BSA_ERR_INVALID_ARG 1  /* null pointer, bad size, inconsistent shapes  */
+#define BSA_ERR_UNSUPPORTED 2  /* valid request outside what the kernels cover */
+#define BSA_ERR_WORKSPACE 3    /* workspace missing or smaller than required   */
+#define BSA_ERR_CUDA 4         /* a CUDA runtime/driver call failed            */
+#define BSA_ERR_DEVICE 5       /* a kernel recorded a fault (see below)        */
+
+/* device error word values (bsa_get_device_error) */
+#define BSA_DEVERR_NONE 0
+#define BSA_DEVERR_BAD_INDEX 1     /* block index outside [0, nKB) or count > max_k */
+#define BSA_DEVERR_TIMEOUT 2       /* a bounded mbarrier wait gave up              */
+#define BSA_DEVERR_SCHEDULE 3      /* a row's KV schedule exceeded the kernel cap  */
+#define BSA_DEVERR_NO_GEOMETRY 4   /* a PARTIAL block met without a fine-mask geometry */
+
+/* ---- per-head modes (DiTFastAttnV2, "Fused Kernel": each head picks full,
+ *      skip with the cached output of the previous step, or arrow) ------- */
+#define BSA_HEAD_FULL 0    /* all KV blocks                              */
+#define BSA_HEAD_SPARSE 1  /* the KV blocks of the block list            */
+#define BSA_HEAD_SKIP 2    /* O = bf16(cache_in), nothing computed       */
+
+/* ---- block classes (bitmap values and block-list flags) ----------------- */
+#define BSA_BLOCK_NONE 0
+#define BSA_BLOCK_FULL 1     /* every real (query, key) pair allowed           */
+#define BSA_BLOCK_PARTIAL 2  /* some pairs allowed: fine mask inside the block */
+
+#define BSA_MASK_ARROW 1
+#define BSA_MASK_GNA 2
+
+#define BSA_SELECT_POOLED_QK 1    /* mean-pooled Q/K block scores              */
+#define BSA_SELECT_FULL_SCORE 2   /* avg-pooled softmax map (SparseD)          */
+
+/* Problem shape. block_q / block_k: tokens per query / key block (the mask
+ * granularity); n_text: text tokens at the front of the sequence. */
+typedef struct {
+  int32_t B, H, N, d;
+  int32_t block_q, block_k;
+  int32_t n_text;
+} bsa_dims;
+
+/* GNA geometry (jsqmd.com GNA article, section 1.1): a 1..3-D token grid
+ * (outermost dimension first), tile extent, window and stride per dimension.
+ * Per dimension of length L, window k and stride s, query i reads keys
+ * [start, start + k) with start = clamp(s*floor(i/s) - s*floor((k-s)/(2s)),
+ * 0, L-k). Tokens are in tile order (see bsa_permute_tiles). */
+typedef struct {
+  int32_t ndim;
+  int32_t grid[3];
+  int32_t tile[3];
+  int32_t window[3];
+  int32_t stride[3];
+} bsa_gna_geom;
+
+typedef struct {
+  int32_t kind;               /* BSA_MASK_ARROW or BSA_MASK_GNA               */
+  const int32_t* head_mode;   /* device int32 [H], BSA_HEAD_*; NULL = all SPARSE */
+  const int32_t* window;      /* device int32 [H], arrow half-width in blocks  */
+  bsa_gna_geom gna;           /* GNA only                                      */
+} bsa_mask_spec;
+
+/* Block list (one row per (b, h, query block)). idx holds the kept KV block
+ * indices in ascending order, padded with -1; flag holds each entry's class
+ * (BSA_BLOCK_FULL / BSA_BLOCK_PARTIAL), padded with 0. bitmap (optional,
+ * NULL to skip) holds the class of every (query block, KV block) pair. */
+typedef struct {
+  int32_t* cnt;     /* device int32 [B, H, nQB]          */
+  int32_t* idx;     /* device int32 [B, H, nQB, max_k]   */
+  uint8_t* flag;    /* device uint8 [B, H, nQB, max_k]   */
+  uint8_t* bitmap;  /* device uint8 [B, H, nQB, nKB] or NULL */
+  int32_t max_k;    /* row capacity, 1 <= max_k          */
+} bsa_block_list;
+
+/* A range [begin, end) of KV blocks whose top-k is cut on its own. */
+typedef struct {
+  int32_t begin, end, k;
+} bsa_key_group;
+
+typedef struct {
+  int32_t method;            /* BSA_SELECT_POOLED_QK or BSA_SELECT_FULL_SCORE */
+  int32_t n_groups;          /* 1..4                                          */
+  bsa_key_group groups[4];
+  int32_t keep_text;         /* 1: text KV blocks always kept, text rows full */
+  float scale;               /* logit scale (FULL_SCORE), usually 1/sqrt(d)   */
+} bsa_select_spec;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int bsa_version(void);
+
+/* Human-readable text of a BSA_* status code (static storage). */
+const char* bsa_error_string(int status);
+
+/* bsa_build_mask: fixed patterns to a block list.
+ *  ARROW (DiTFastAttnV2, "Head-wise Arrow Attention" and "Fused Kernel"):
+ *    block (I, J) is kept iff I or J holds a text token or |I - J| <= w_h;
+ *    kept blocks are dense (FULL). Needs block_q == block_k.
+ *  GNA (jsqmd.com GNA article, sections 1.1 and 2.1): tile-order tokens,
+ *    block size == tile volume; a (Q tile, KV tile) pair is FULL when every
+ *    real pair is inside the window, PARTIAL when some are, dropped when none
+ *    are; text rows and columns are full; padded tokens are never keys.
+ *  FULL heads keep every block, SKIP heads keep none (cnt = 0).
+ *  Writes cnt, idx, flag (and bitmap if non-NULL) for all B*H*nQB rows.
+ *  Errors: INVALID_ARG (null pointers, max_k < nKB, bad geometry),
+ *  UNSUPPORTED (arrow with block_q != block_k; GNA with tile x-extent that is
+ *  neither a divisor nor a multiple of 64, or block size != tile volume). */
+int bsa_build_mask(const bsa_dims* dims, const bsa_mask_spec* spec,
+                   const bsa_block_list* out, void* stream);
+
+/* Workspace bytes bsa_select_topk needs for these dims and spec. */
+size_t bsa_select_workspace_size(const bsa_dims* dims, const bsa_select_spec* spec);
+
+/* bsa_select_topk: content-driven block selection.
+ *  POOLED_QK (lmnt.cn BSA post, sections 2.2-2.3): each block is mean-pooled
+ *    (fp32, ragged last block over its real tokens); score(I,J) = Qbar_I .
+ *    Kbar_J in fp32; each group keeps its top k by descending score, ties to
+ *    the lower index. keep_text: text KV blocks always kept (not counted in
+ *    k) and text query rows keep every block.
+ *  FULL_SCORE (SparseD, "Isolated Selection"): A = softmax(scale*QK^T + bias)
+ *    over all keys, A' = avgpool(A, block); each group (e.g. prefill and
+ *    generation key blocks) keeps its own top k per query block.
+ *  block_bias: optional device fp32 [H, nQB, nKB] logit offset (FULL_SCORE).
+ *  Writes the block list (all entries FULL). Workspace: device, at least
+ *  bsa_select_workspace_size bytes, 256-byte aligned; contents are scratch.
+ *  Errors: INVALID_ARG, UNSUPPORTED (d not 64/128, FULL_SCORE with block size
+ *  not a multiple of 128 or block_q != block_k), WORKSPACE. */
+int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K,
+                    const bsa_select_spec* spec, const float* block_bias,
+                    void* workspace, size_t workspace_bytes,
+                    const bsa_block_list* out, void* stream);
+
+/* bsa_forward: FlashAttention-style forward over the kept blocks only
+ * (lmnt.cn BSA post, section 3.1: tiles, online softmax, a block-index
+ * variant; DiTFastAttnV2 "Fused Kernel": three per-head modes).
+ *  For each (b, h): SKIP -> O = bf16(cache_in), round to nearest even.
+ *  Otherwise each query row attends the keys of its kept blocks:
+ *    z = scale * q.k + bias(I, J); o = softmax(z) V, fp32 accumulation,
+ *    O rounded to bf16; PARTIAL blocks apply the GNA fine mask from `gna`.
+ *  A row with no kept key gives 0.
+ *  head_mode: device int32 [H]. list: needed when any head is SPARSE.
+ *  gna: host struct, NULL unless the list has PARTIAL blocks or the tile
+ *  layout has padding. cache_in: device fp32 [B,H,N,d], needed when any head
+ *  is SKIP. cache_out: NULL or device fp32 [B,H,N,d]; receives the fp32
+ *  output of computed heads (SKIP heads are not written).
+ *  block_bias: NULL or device fp32 [H, nQB, nKB], natural-log units.
+ *  Errors: INVALID_ARG, UNSUPPORTED (d not 64/128, block sizes not multiples
+ *  of 64, N > 131072), CUDA. */
+int bsa_forward(const bsa_dims* dims, const void* Q, const void* K, const void* V,
+                const bsa_block_list* list, const int32_t* head_mode,
+                const bsa_gna_geom* gna, const float* cache_in, float* cache_out,
+                const float* block_bias, float scale, void* O, void* stream);
+
+/* Length of the tile-order sequence for a raster sequence of n_text text
+ * tokens plus the GNA grid: text padded to a multiple of the tile volume,
+ * plus every (padded) tile. Host only. */
+int bsa_gna_tiled_len(int32_t n_text, const bsa_gna_geom* geom, int32_t* n_tiled);
+
+/* bsa_permute_tiles / bsa_unpermute_tiles (jsqmd.com GNA article, section
+ * 2.2: token permutation fused with padding in one copy kernel).
+ *  permute: `in[t]` raster [B, H, n_text + prod(grid), d] bf16 ->
+ *    `out[t]` tile order [B, H, n_tiled, d] bf16, padding rows zeroed.
+ *  unpermute: the inverse; padding rows are dropped.
+ *  dims: B, H, d and n_text are read (N and block sizes are ignored).
+ *  in/out: HOST arrays of n_tensors (1..4) device pointers.
+ *  Errors: INVALID_ARG, UNSUPPORTED (d not a multiple of 8). */
+int bsa_permute_tiles(const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_tensors,
+                      const void* const* in, void* const* out, void* stream);
+int bsa_unpermute_tiles(const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_tensors,
+                        const void* const* in, void* const* out, void* stream);
+
+/* Synchronise `stream`, then read and clear the device error word.
+ * *code receives a BSA_DEVERR_* value. Returns BSA_OK, or BSA_ERR_CUDA if the
+ * synchronisation itself failed. */
+int bsa_get_device_error(void* stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H */
