@@ -166,7 +166,8 @@ def gna_block_classes_separable(lay: GnaLayout):
     """
     nB = lay.ntb + lay.n_tiles
     out = np.zeros((nB, nB), dtype=np.uint8)
-    text_pad = lay.text_span > lay.n_text
+    # only a text block reaching past n_text holds padding slots
+    text_pad = [(J + 1) * lay.bs > lay.n_text for J in range(lay.ntb)]
     tiles = [np.unravel_index(t, lay.tiles) for t in range(lay.n_tiles)]
     rng = []
     for tc in tiles:
@@ -180,7 +181,7 @@ def gna_block_classes_separable(lay: GnaLayout):
     for I in range(nB):
         for J in range(nB):
             if I < lay.ntb or J < lay.ntb:
-                k_pad = text_pad if J < lay.ntb else padded_tile[J - lay.ntb]
+                k_pad = text_pad[J] if J < lay.ntb else padded_tile[J - lay.ntb]
                 out[I, J] = BLOCK_PARTIAL if k_pad else BLOCK_FULL
                 continue
             rq, rk = rng[I - lay.ntb], rng[J - lay.ntb]

@@ -94,6 +94,8 @@ def _layouts():
     yield M.GnaLayout(4, (6, 7), (2, 4), (3, 4), (1, 2))
     yield M.GnaLayout(3, (4, 6, 5), (2, 2, 4), (2, 3, 3), (1, 1, 1))
     yield M.GnaLayout(8, (4, 6, 8), (2, 2, 2), (2, 4, 4), (2, 2, 2))
+    yield M.GnaLayout(20, (4, 6), (2, 4), (3, 3), (1, 1))   # three text blocks, the last padded
+    yield M.GnaLayout(16, (3, 5), (2, 4), (3, 2), (1, 2))   # text ends on a block edge
 
 
 @pytest.mark.parametrize("lay", list(_layouts()))
