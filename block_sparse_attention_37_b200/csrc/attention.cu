@@ -65,16 +65,20 @@ __device__ __forceinline__ void cta_fail(volatile int* abort_flag, int code) {
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
 __device__ __forceinline__ uint32_t bit_range(int a, int b) {  // bits [a, b) of a 32-bit word
+  a = max(a, 0);
+  b = min(b, 32);
   if (a >= b) return 0u;
   const uint32_t hi = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
-  const uint32_t lo = a <= 0 ? 0u : ((1u << a) - 1u);
+  const uint32_t lo = (1u << a) - 1u;
   return hi & ~lo;
 }
 
-__device__ __forceinline__ uint64_t bit_range64(int a, int b) {
+__device__ __forceinline__ uint64_t bit_range64(int a, int b) {  // bits [a, b), clipped to [0, 64)
+  a = max(a, 0);
+  b = min(b, 64);
   if (a >= b) return 0ull;
   const uint64_t hi = b >= 64 ? ~0ull : ((1ull << b) - 1ull);
-  const uint64_t lo = a <= 0 ? 0ull : ((1ull << a) - 1ull);
+  const uint64_t lo = (1ull << a) - 1ull;
   return hi & ~lo;
 }
 

@@ -203,7 +203,7 @@ def _gna_forward(B, H, n_text, grid, tile, window, stride, d, seed, modes, rows_
     (64, (4, 8, 16), (2, 4, 8), (3, 5, 7), (1, 1, 1)),      # partial tiles everywhere
     (50, (5, 9, 20), (2, 4, 8), (3, 5, 7), (1, 2, 2)),      # padding in grid and text
     (0, (300,), (64,), (97,), (5,)),                          # 1-D, padded last tile
-    (128, (8, 16), (1, 128), (3, 48), (1, 16)),               # x tile wider than a segment
+    (128, (8, 256), (1, 128), (3, 48), (1, 16)),              # x tile wider than a segment
 ])
 def test_forward_gna_small(n_text, grid, tile, window, stride):
     _gna_forward(1, 3, n_text, grid, tile, window, stride, 128, 7, modes=[1, 0, 1])
