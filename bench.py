@@ -355,6 +355,27 @@ CONFIGS = {
 DEFAULT_SEEDS = {"c1": 0, "c2": 1, "c3": 2, "c4": 3, "c5s": 4, "c5f": 4}
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def rank_seed(cfg: str, rank: int) -> int:
+    """Seed of rank `rank`'s independent instance (weak scaling: every rank owns its own batch)."""
+    return DEFAULT_SEEDS[cfg] + 1000 * rank
+
+
+def reduce_max(vals, world: int, device) -> list:
+    """Element-wise max over ranks (timing only; the data path has no collective)."""
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_throughput(flops_per_step: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: the units all ranks processed over the slowest rank's time."""
+    return flops_per_step * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- timing
 
 def time_steps(job, steps, warmup, flush, with_fwd_events=True):
@@ -450,7 +471,7 @@ def run_bsa(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     cfg = args.config
     desc, make, JobT = CONFIGS[cfg]
-    seed = DEFAULT_SEEDS[cfg] + 1000 * rank
+    seed = rank_seed(cfg, rank)
     w = make(seed)
     job = JobT(w)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
@@ -467,14 +488,10 @@ def run_bsa(args, rank, world, local_rank):
     sampler.stop()
     if world > 1:
         dist.barrier()
-    total_ms = float(np.sum(step_ms))
-    t = torch.tensor([total_ms, float(np.sum(fwd_ms))], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_total = float(t[0]), float(t[1])
+    total_ms, fwd_total = reduce_max([np.sum(step_ms), np.sum(fwd_ms)], world, "cuda")
     ms_per_step = total_ms / args.steps
     fwd_ms_mean = fwd_total / args.steps
-    value = job.flops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(job.flops, world, ms_per_step)
 
     extra = {}
     if not args.no_dense:
@@ -503,13 +520,10 @@ def run_bsa(args, rank, world, local_rank):
             job.e2e_step()
         e1.record()
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1) / n
-        te = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": job.flops * world / (float(te[0]) * 1e-3) / 1e12, "unit": UNIT,
+        (e2e_ms,) = reduce_max([e0.elapsed_time(e1) / n], world, "cuda")
+        e2e = {"value": job_throughput(job.flops, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": int(job.h2d), "d2h_bytes_per_step": int(job.d2h),
-               "ms_per_step": float(te[0])}
+               "ms_per_step": e2e_ms}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
