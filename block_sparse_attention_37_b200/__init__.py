@@ -26,8 +26,9 @@ SELECT_POOLED_QK, SELECT_FULL_SCORE = 1, 2
 EXPORTS = (
     "bsa_version", "bsa_error_string", "bsa_build_mask", "bsa_select_workspace_size",
     "bsa_select_topk", "bsa_forward", "bsa_gna_tiled_len", "bsa_permute_tiles",
-    "bsa_unpermute_tiles", "bsa_get_device_error",
+    "bsa_unpermute_tiles", "bsa_get_device_error", "bsa_select_topk_static",
 )
+STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class BsaError(RuntimeError):
@@ -102,6 +103,7 @@ def _lib():
         lib.bsa_permute_tiles.argtypes = [P, P, ctypes.c_int32, P, P, P]
         lib.bsa_unpermute_tiles.argtypes = [P, P, ctypes.c_int32, P, P, P]
         lib.bsa_get_device_error.argtypes = [P, P]
+        lib.bsa_select_topk_static.argtypes = [P, P, P, P, P, P, P]
         _LIB = lib
     return _LIB
 
@@ -205,6 +207,15 @@ def select_topk(dm: Dims, q, k, spec: SelectSpec, out: BlockList, workspace, bia
                                   ctypes.byref(spec), _ptr(bias, torch.float32, "bias"),
                                   _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
                                   ctypes.byref(lc), _stream(stream)), "bsa_select_topk")
+
+
+def select_topk_static(dm: Dims, q, k, spec: SelectSpec, out: BlockList, bias=None, stream=None):
+    """bsa_select_topk_static: selection with the library's fixed scratch (no allocation)."""
+    lc = out.c()
+    _check(_lib().bsa_select_topk_static(ctypes.byref(dm), _ptr(q, torch.bfloat16, "Q"),
+                                         _ptr(k, torch.bfloat16, "K"), ctypes.byref(spec),
+                                         _ptr(bias, torch.float32, "bias"), ctypes.byref(lc), _stream(stream)),
+           "bsa_select_topk_static")
 
 
 def forward(dm: Dims, q, k, v, o, head_mode, blocks: BlockList | None = None, gna: GnaGeom | None = None,

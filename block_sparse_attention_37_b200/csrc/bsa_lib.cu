@@ -5,3 +5,4 @@
 #include "mask.cu"
 #include "permute.cu"
 #include "select.cu"
+#include "select_static.cu"

@@ -156,6 +156,33 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K,
                     void* workspace, size_t workspace_bytes,
                     const bsa_block_list* out, void* stream);
 
+/* Size of the library-owned scratch behind bsa_select_topk_static: 16 MiB,
+ * enough for the pooled selection at 24 heads x 16896 tokens (3.2 MB) and the
+ * full-score selection at 32 heads x 32768 tokens (12 MB). */
+#define BSA_STATIC_SCRATCH_BYTES (16u << 20)
+
+/* bsa_select_topk_static: bsa_select_topk without a caller workspace. The
+ * pages have no counterpart; this entry point exists for callers that cannot
+ * allocate device memory at call time - runtimes that plan every device
+ * buffer ahead in a fixed arena, or latency-critical loops that must not
+ * call cudaMalloc (which can synchronise the device) - but still own Q, K
+ * and the block list.
+ *  Same arguments and results as bsa_select_topk, minus the workspace. The
+ *  scratch is a fixed BSA_STATIC_SCRATCH_BYTES array inside the library; every
+ *  GPU that loads the library holds it until the process exits. Nothing is
+ *  allocated: no cudaMalloc, no cudaFree, no allocating library call.
+ *  The first call on a device looks up the array's device address
+ *  (cudaGetSymbolAddress) with that device current; make that first call
+ *  before any stream capture on the device.
+ *  All calls share the one array, which keeps the previous call's contents
+ *  (the kernels clear what must start at zero). Calls whose kernels overlap on
+ *  the GPU (e.g. on two streams) race on the scratch: serialise them.
+ *  Errors: those of bsa_select_topk, and BSA_ERR_WORKSPACE when
+ *  bsa_select_workspace_size(dims, spec) exceeds BSA_STATIC_SCRATCH_BYTES. */
+int bsa_select_topk_static(const bsa_dims* dims, const void* Q, const void* K,
+                           const bsa_select_spec* spec, const float* block_bias,
+                           const bsa_block_list* out, void* stream);
+
 /* bsa_forward: FlashAttention-style forward over the kept blocks only
  * (lmnt.cn BSA post, section 3.1: tiles, online softmax, a block-index
  * variant; DiTFastAttnV2 "Fused Kernel": three per-head modes).
