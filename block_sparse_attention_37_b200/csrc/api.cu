@@ -286,10 +286,10 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K, const bs
     ap.lse = reinterpret_cast<float*>(ws + L.lse);
     ap.apool = reinterpret_cast<float*>(ws + L.apool);
     const int grid = (int)(BH * ap.nQT);
-    if ((st = cuda_status(launch_attention(dims->d, KIND_LSE, mq, mk, mk, ap, grid, s))) != BSA_OK) return st;
+    if ((st = cuda_status(launch_score(dims->d, KIND_LSE, mq, mk, ap, grid, s))) != BSA_OK) return st;
     if ((st = cuda_status(cudaMemsetAsync(ap.apool, 0, (size_t)BH * nQB * nKB * sizeof(float), s))) != BSA_OK)
       return st;
-    if ((st = cuda_status(launch_attention(dims->d, KIND_POOL, mq, mk, mk, ap, grid, s))) != BSA_OK) return st;
+    if ((st = cuda_status(launch_score(dims->d, KIND_POOL, mq, mk, ap, grid, s))) != BSA_OK) return st;
     sp.apool = ap.apool;
   }
   return cuda_status(launch_select(dims->d, sp, s));
@@ -320,10 +320,11 @@ int bsa_forward(const bsa_dims* dims, const void* Q, const void* K, const void* 
     ap.has_gna = 1;
   }
   const long long BH = (long long)dims->B * dims->H;
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if ((st = make_map(&mq, Q, BH, dims->N, dims->d)) != BSA_OK) return st;
   if ((st = make_map(&mk, K, BH, dims->N, dims->d)) != BSA_OK) return st;
   if ((st = make_map(&mv, V, BH, dims->N, dims->d)) != BSA_OK) return st;
+  if ((st = make_map(&mo, O, BH, dims->N, dims->d)) != BSA_OK) return st;
   ap.B = dims->B;
   ap.H = dims->H;
   ap.N = dims->N;
@@ -346,9 +347,9 @@ int bsa_forward(const bsa_dims* dims, const void* Q, const void* K, const void* 
   ap.bias = block_bias;
   ap.scale_log2 = scale * 1.4426950408889634f;
   ap.O = static_cast<__nv_bfloat16*>(O);
-  const long long grid = BH * ap.nQT;
+  const long long grid = BH * ceil_div(dims->N, 256);
   if (grid > 0x7fffffffll) return BSA_ERR_UNSUPPORTED;
-  return cuda_status(launch_attention(dims->d, KIND_FWD, mq, mk, mv, ap, (int)grid, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_forward(dims->d, mq, mk, mv, mo, ap, (int)grid, static_cast<cudaStream_t>(stream)));
 }
 
 static int permute_common(bool forward, const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_tensors,

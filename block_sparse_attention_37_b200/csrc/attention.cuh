@@ -1,11 +1,11 @@
-// Parameters and launcher of the tcgen05 attention kernel (attention.cu).
+// Parameters and launchers of the tcgen05 attention kernels (forward.cu, score.cu).
 #pragma once
 
 #include "common.cuh"
 
 namespace bsa {
 
-enum { KIND_FWD = 0, KIND_LSE = 1, KIND_POOL = 2 };
+enum { KIND_LSE = 1, KIND_POOL = 2 };
 
 // 64-key segments per sequence the per-CTA schedule can hold: N <= 131072.
 constexpr int kMaxSeg = 2048;
@@ -32,7 +32,12 @@ struct AttnParams {
   GnaDev g;
 };
 
-cudaError_t launch_attention(int d, int kind, const CUtensorMap& q, const CUtensorMap& k,
-                             const CUtensorMap& v, const AttnParams& p, int grid, cudaStream_t stream);
+// The forward: two 128-row query tiles per CTA (forward.cu); grid = B*H*ceil(N/256).
+cudaError_t launch_forward(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                           const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream);
+
+// The two score passes of the full-score selection (score.cu); grid = B*H*ceil(N/128).
+cudaError_t launch_score(int d, int kind, const CUtensorMap& q, const CUtensorMap& k, const AttnParams& p,
+                         int grid, cudaStream_t stream);
 
 }  // namespace bsa

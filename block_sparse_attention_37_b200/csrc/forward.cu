@@ -1,0 +1,724 @@
+// The block-sparse forward (bsa_forward) on sm_100a, two query tiles per CTA.
+//
+// A CTA owns 256 query rows of one (b, h): two 128-row tiles, one per softmax
+// warpgroup. The key side is the union, over the four 64-row groups, of the
+// kept 64-key segments, with one validity bit per group; a warpgroup skips a
+// 128-key tile none of its rows keeps, so each tile costs tensor work only
+// for the warpgroups that need it while K and V are loaded once.
+// Roles (320 threads):
+//   warp 0     TMA producer: both Q tiles, then K/V tiles into a shared ring
+//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2-5  softmax warpgroup 0 (rows 0..127 of the CTA)
+//   warps 6-9  softmax warpgroup 1 (rows 128..255)
+// Tensor memory (512 columns): S/P of warpgroup w at column 128w, O of
+// warpgroup w at 256 + w*D. The MMA warp alternates the two warpgroups, so
+// the tensor core runs one group's PV and next QK^T while the other group's
+// softmax runs (lmnt.cn BSA post, section 3.1: FlashAttention tiles with
+// online softmax over the selected blocks; DiTFastAttnV2 "Fused Kernel").
+// Output leaves through shared memory and a TMA store.
+#include "tiles.cuh"
+
+namespace bsa {
+
+constexpr float kRescaleTau = 8.0f;  // O is rescaled only when the row max grows by more than 2^8
+
+template <int D>
+struct FwdCfg {
+  static constexpr int STAGES = D == 64 ? 4 : 2;
+  static constexpr int TILE = 128 * D * 2;
+  static constexpr int CHUNK = 128 * 128;  // 128 rows x 64 bf16
+  static constexpr int Q_OFF = 0;          // two Q tiles (reused as O staging)
+  static constexpr int K_OFF = 2 * TILE;
+  static constexpr int V_OFF = K_OFF + STAGES * TILE;
+  static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
+  static constexpr int NBAR = 2 + 4 * STAGES + 6;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int BITS_OFF = MISC_OFF + 64;
+  static constexpr int SCHED_OFF = BITS_OFF + 5 * 64 * 4;
+  static constexpr int SMEM_BYTES = SCHED_OFF + kMaxSeg * 4;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+};
+static_assert(FwdCfg<128>::SMEM_ALLOC <= 227 * 1024, "smem budget");
+static_assert(FwdCfg<64>::SMEM_ALLOC <= 227 * 1024, "smem budget");
+
+// Segment entry bits: index in [0, 24), group-valid bits g0..g3 at 24..27, partial at 28.
+constexpr int kGrpShift = 24;
+constexpr int kPart4 = 1 << 28;
+
+__device__ __forceinline__ void named_bar(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* src, int c0, int c1, int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(m)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (x0, x1) * c + (o, o), two lanes in one instruction
+__device__ __forceinline__ void fma2(float& x0, float& x1, float c, float o) {
+  uint64_t v, cc, oo;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(oo) : "f"(o));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(v), "l"(cc), "l"(oo));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(v));
+}
+
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  uint64_t a, b;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(a) : "l"(a), "l"(b));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
+}
+
+// 2^x on the FMA pipe, two lanes at a time, to take load off the MUFU unit
+// (16 ex2/clk/SM). Range reduction x = j + f with j = round(x) (added to the
+// exponent field) and f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted
+// for minimum relative error on that interval (max relative error 7.5e-5,
+// below the bf16 rounding of P). x is clamped at -127, where the result is
+// exactly 0 (see below), so masked (-inf) entries give 0 as on the MUFU path.
+constexpr float kExpC0 = 0.9999280571937561f;
+constexpr float kExpC1 = 0.6932609677314758f;
+constexpr float kExpC2 = 0.2426111400127411f;
+constexpr float kExpC3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ void poly_exp2_2(float& x0, float& x1) {
+  x0 = fmaxf(x0, -127.f);
+  x1 = fmaxf(x1, -127.f);
+  uint64_t x, t, j, f, p, c;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(kRoundMagic));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(c));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(j) : "l"(t), "l"(c));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(j));
+  uint64_t c3, c2, c1, c0;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c3) : "f"(kExpC3));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(kExpC2));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c1) : "f"(kExpC1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(c0) : "f"(kExpC0));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c0));
+  uint32_t t0, t1, p0, p1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
+  p0 = t0 * 8388608u + p0;  // j << 23 added to the exponent bits
+  p1 = t1 * 8388608u + p1;
+  // At x = -127 (every masked key) p(0) = kExpC0 < 1, so the exponent
+  // underflows into the sign bit; the signed max turns that into exactly 0.
+  x0 = __int_as_float(max((int)p0, 0));
+  x1 = __int_as_float(max((int)p1, 0));
+}
+
+// Of every 8 exponent pairs of a row, how many go to the FMA pipe.
+constexpr int kEmuPairsPer8 = 2;
+
+// Fill one group's segment bits from a block-list row.
+__device__ void fill_group_bits(const AttnParams& p, size_t row, uint32_t* vb, uint32_t* pb, int lane) {
+  const int spb = p.block_k >> 6;
+  int n = p.cnt[row];
+  if (n < 0 || n > p.max_k) {
+    if (lane == 0) record_error(BSA_DEVERR_BAD_INDEX);
+    n = n < 0 ? 0 : p.max_k;
+  }
+  const int32_t* ip = p.idx + row * p.max_k;
+  const uint8_t* fp = p.flag + row * p.max_k;
+  for (int e = lane; e < n; e += 32) {
+    const int J = ip[e];
+    if (J < 0 || J >= p.nKB) {
+      record_error(BSA_DEVERR_BAD_INDEX);
+      continue;
+    }
+    bool part = fp[e] == BSA_BLOCK_PARTIAL;
+    if (part && !p.has_gna) {
+      record_error(BSA_DEVERR_NO_GEOMETRY);
+      part = false;
+    }
+    for (int u = 0; u < spb; ++u) {
+      const int s = J * spb + u;
+      if (s >= p.nSeg) break;
+      atomicOr(&vb[s >> 5], 1u << (s & 31));
+      if (part) atomicOr(&pb[s >> 5], 1u << (s & 31));
+    }
+  }
+}
+
+// Sorted union schedule of the CTA's four 64-row groups (warp 0). Returns count.
+__device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0, uint32_t* vb,
+                                 uint32_t* pb, int32_t* sched, int lane) {
+  const int nwords = (p.nSeg + 31) >> 5;
+  for (int w = lane; w < 5 * 64; w += 32) vb[w] = 0u;  // vb[4][64] then pb[64]
+  __syncwarp();
+  bool valid[4];
+  int I[4];
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    valid[g] = row0 + 64 * g < p.N;
+    I[g] = valid[g] ? (row0 + 64 * g) / p.block_q : -1;
+  }
+  const int spb = p.block_k >> 6;
+  if (mode == BSA_HEAD_FULL) {
+    for (int w = lane; w < nwords; w += 32) vb[w] = bit_range(0, min(32, p.nSeg - w * 32));
+    if (p.has_gna && p.g.has_padding)
+      for (int J = lane; J < p.nKB; J += 32) {
+        if (!gna_block_padded(p.g, J)) continue;
+        for (int u = 0; u < spb; ++u) {
+          const int s = J * spb + u;
+          if (s < p.nSeg) atomicOr(&pb[s >> 5], 1u << (s & 31));
+        }
+      }
+    __syncwarp();
+    for (int g = 1; g < 4; ++g)
+      for (int w = lane; w < 64; w += 32) vb[g * 64 + w] = vb[w];
+  } else {
+    if (p.cnt == nullptr) {
+      if (lane == 0) record_error(BSA_DEVERR_BAD_INDEX);
+    } else {
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        if (valid[g] && (g == 0 || I[g] != I[g - 1]))
+          fill_group_bits(p, (size_t)bh * p.nQB + I[g], vb + g * 64, pb, lane);
+    }
+    __syncwarp();
+    // groups sharing a query block share its bits; groups past N copy their neighbour
+    for (int g = 1; g < 4; ++g) {
+      if (!valid[g] || I[g] == I[g - 1])
+        for (int w = lane; w < 64; w += 32) vb[g * 64 + w] = vb[(g - 1) * 64 + w];
+      __syncwarp();
+    }
+  }
+  __syncwarp();
+  const int w0 = lane, w1 = lane + 32;
+  uint32_t a0 = 0u, a1 = 0u;
+  if (w0 < nwords) a0 = vb[w0] | vb[64 + w0] | vb[128 + w0] | vb[192 + w0];
+  if (w1 < nwords) a1 = vb[w1] | vb[64 + w1] | vb[128 + w1] | vb[192 + w1];
+  const int c0 = __popc(a0), c1 = __popc(a1);
+  int i0 = c0, i1 = c1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t0 = __shfl_up_sync(0xffffffffu, i0, o);
+    const int t1 = __shfl_up_sync(0xffffffffu, i1, o);
+    if (lane >= o) {
+      i0 += t0;
+      i1 += t1;
+    }
+  }
+  const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
+  const int tot1 = __shfl_sync(0xffffffffu, i1, 31);
+  int off = i0 - c0;
+  for (uint32_t a = a0; a; a &= a - 1) {
+    const int b = __ffs(a) - 1;
+    int e = w0 * 32 + b;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) e |= ((vb[g * 64 + w0] >> b) & 1u) << (kGrpShift + g);
+    if ((pb[w0] >> b) & 1u) e |= kPart4;
+    sched[off++] = e;
+  }
+  off = tot0 + i1 - c1;
+  for (uint32_t a = a1; a; a &= a - 1) {
+    const int b = __ffs(a) - 1;
+    int e = w1 * 32 + b;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) e |= ((vb[g * 64 + w1] >> b) & 1u) << (kGrpShift + g);
+    if ((pb[w1] >> b) & 1u) e |= kPart4;
+    sched[off++] = e;
+  }
+  return tot0 + tot1;
+}
+
+// Bit w of the result: does warpgroup w need tile t?
+__device__ __forceinline__ int tile_need(const int32_t* sched, int nseg, int t, int act_mask) {
+  const int ea = sched[2 * t];
+  const int eb = (2 * t + 1 < nseg) ? sched[2 * t + 1] : 0;
+  const int g = ((ea | eb) >> kGrpShift) & 0xF;
+  return (((g & 3) ? 1 : 0) | ((g & 12) ? 2 : 0)) & act_mask;
+}
+
+template <int D>
+__device__ void skip_copy256(const AttnParams& p, int bh, int row0) {
+  if (p.cache_in == nullptr) {
+    if (threadIdx.x == 0) record_error(BSA_DEVERR_BAD_INDEX);
+    return;
+  }
+  const int rows = min(256, p.N - row0);
+  const size_t base = ((size_t)bh * p.N + row0) * D;
+  const float4* src = reinterpret_cast<const float4*>(p.cache_in + base);
+  uint2* dst = reinterpret_cast<uint2*>(p.O + base);
+  const int n4 = rows * D / 4;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) {
+    const float4 v = __ldg(src + i);
+    uint2 o;
+    o.x = pack_bf16x2(v.x, v.y);
+    o.y = pack_bf16x2(v.z, v.w);
+    dst[i] = o;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const AttnParams p) {
+  using C = FwdCfg<D>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nQP = (p.N + 255) >> 8;
+  const int work = p.order ? p.order[blockIdx.x] : (int)blockIdx.x;
+  const int pair = work % nQP;
+  const int bh = work / nQP;
+  const int h = bh % p.H;
+  const int row0 = pair * 256;
+
+  const int mode = p.head_mode[h];
+  if (mode < BSA_HEAD_FULL || mode > BSA_HEAD_SKIP) {
+    if (tid == 0) record_error(BSA_DEVERR_BAD_INDEX);
+    return;
+  }
+  if (mode == BSA_HEAD_SKIP) {
+    skip_copy256<D>(p, bh, row0);
+    return;
+  }
+
+  uint8_t* sQ = smem + C::Q_OFF;
+  uint8_t* sK = smem + C::K_OFF;
+  uint8_t* sV = smem + C::V_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars;          // [2]
+  uint64_t* k_full = bars + 2;      // [S]
+  uint64_t* k_empty = k_full + S;   // [S]
+  uint64_t* v_full = k_empty + S;   // [S]
+  uint64_t* v_empty = v_full + S;   // [S]
+  uint64_t* s_full = v_empty + S;   // [2]
+  uint64_t* p_full = s_full + 2;    // [2]
+  uint64_t* o_ready = p_full + 2;   // [2]
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  uint32_t* vb = reinterpret_cast<uint32_t*>(smem + C::BITS_OFF);
+  int32_t* sched = reinterpret_cast<int32_t*>(smem + C::SCHED_OFF);
+
+  if (tid == 0) {
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&q_full[w], 1);
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w], 128);
+      mbar_init(&o_ready[w], 1);
+    }
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(misc, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0) {
+    const int n = build_schedule256(p, mode, bh, row0, vb, vb + 256, sched, lane);
+    // tiles each warpgroup needs
+    const int act = 1 | ((row0 + 128 < p.N) ? 2 : 0);
+    const int T = (n + 1) >> 1;
+    int c0 = 0, c1 = 0;
+    for (int t = lane; t < T; t += 32) {
+      const int nw = tile_need(sched, n, t, act);
+      c0 += nw & 1;
+      c1 += nw >> 1;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      c0 += __shfl_xor_sync(0xffffffffu, c0, o);
+      c1 += __shfl_xor_sync(0xffffffffu, c1, o);
+    }
+    if (lane == 0) {
+      misc[2] = n;
+      misc[3] = c0;
+      misc[4] = c1;
+      misc[5] = act;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+  const int nseg = (int)misc[2];
+  const int T = (nseg + 1) >> 1;
+  const int act = (int)misc[5];
+  const int wg_tiles0 = (int)misc[3], wg_tiles1 = (int)misc[4];
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0 && T > 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+#pragma unroll
+      for (int w = 0; w < 2; ++w) {
+        if ((w ? wg_tiles1 : wg_tiles0) == 0) continue;
+        mbar_arrive_expect_tx(&q_full[w], C::TILE);
+        for (int c = 0; c < D / 64; ++c)
+          for (int r = 0; r < 2; ++r)
+            tma_load_3d(sQ + w * C::TILE + c * C::CHUNK + r * (C::CHUNK / 2), &tmQ, &q_full[w], c * 64,
+                        row0 + 128 * w + 64 * r, bh);
+      }
+      int k_issued = 0, v_issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % S;
+        const uint32_t ph = (uint32_t)(t / S) & 1u;
+        const int sa = sched[2 * t] & kSegIdxMask;
+        const int sb = (2 * t + 1 < nseg) ? (sched[2 * t + 1] & kSegIdxMask) : sa;
+        if (t >= S && !mbar_wait(&k_empty[st], ph ^ 1u, abort_flag)) {
+          cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&k_full[st], C::TILE);
+        uint8_t* dk = sK + st * C::TILE;
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(dk + c * C::CHUNK, &tmK, &k_full[st], c * 64, sa * 64, bh);
+          tma_load_3d(dk + c * C::CHUNK + C::CHUNK / 2, &tmK, &k_full[st], c * 64, sb * 64, bh);
+        }
+        k_issued = t + 1;
+        if (t >= S && !mbar_wait(&v_empty[st], ph ^ 1u, abort_flag)) {
+          cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[st], C::TILE);
+        uint8_t* dv = sV + st * C::TILE;
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(dv + c * C::CHUNK, &tmV, &v_full[st], c * 64, sa * 64, bh);
+          tma_load_3d(dv + c * C::CHUNK + C::CHUNK / 2, &tmV, &v_full[st], c * 64, sb * 64, bh);
+        }
+        v_issued = t + 1;
+      }
+      if (*abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        auto drain = [&](uint64_t* bar, uint32_t ph) {
+          while (!mbar_try_wait(smem_u32(bar), ph) && globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+        };
+        if (wg_tiles0 > 0) drain(&q_full[0], 0u);
+        if (wg_tiles1 > 0) drain(&q_full[1], 0u);
+        for (int t = k_issued - S < 0 ? 0 : k_issued - S; t < k_issued; ++t)
+          drain(&k_full[t % S], (uint32_t)(t / S) & 1u);
+        for (int t = v_issued - S < 0 ? 0 : v_issued - S; t < v_issued; ++t)
+          drain(&v_full[t % S], (uint32_t)(t / S) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+      bool ok = true;
+      // per-warpgroup state in scalars (no local memory on the issue path)
+      int pend0 = -1, pend1 = -1;  // tile whose PV is still to be issued
+      int done0 = 0, done1 = 0;    // QK^T tiles issued
+      uint32_t q_ok = 0u;          // bit w: Q tile w has landed
+      uint32_t v_left = 0u;        // 2 bits per stage: PVs still to read that stage's V
+      auto do_pv = [&](int w) -> bool {
+        const int u = w ? pend1 : pend0;
+        const int j = (w ? done1 : done0) - 1;
+        const int st = u % S;
+        if (!mbar_wait(&p_full[w], (uint32_t)j & 1u, abort_flag)) return false;
+        if (!mbar_wait(&v_full[st], (uint32_t)(u / S) & 1u, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vbase = sVa + st * C::TILE;
+        const uint32_t ptm = tmem + w * 128, otm = tmem + 256 + w * D;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(otm, ptm + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::CHUNK, 1024), idesc_pv,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&o_ready[w]);
+        const uint32_t left = ((v_left >> (2 * st)) & 3u) - 1u;
+        v_left = (v_left & ~(3u << (2 * st))) | (left << (2 * st));
+        if (left == 0) tc_commit(&v_empty[st]);
+        if (w) pend1 = -1; else pend0 = -1;
+        return true;
+      };
+      auto do_qk = [&](int w, int t, uint32_t kbase) -> bool {
+        if (!((q_ok >> w) & 1u)) {
+          if (!mbar_wait(&q_full[w], 0u, abort_flag)) return false;
+          tc_fence_after();
+          q_ok |= 1u << w;
+        }
+        if ((w ? pend1 : pend0) >= 0 && !do_pv(w)) return false;
+        const uint32_t qbase = sQa + w * C::TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
+          umma_ss(tmem + w * 128, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                  idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[w]);
+        if (w) {
+          pend1 = t;
+          ++done1;
+        } else {
+          pend0 = t;
+          ++done0;
+        }
+        return true;
+      };
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t % S;
+        // a PV still pending on this stage is issued before the stage is reused
+        if (pend0 >= 0 && pend0 % S == st) ok = do_pv(0);
+        if (ok && pend1 >= 0 && pend1 % S == st) ok = do_pv(1);
+        if (!ok) break;
+        const int nw = tile_need(sched, nseg, t, act);
+        ok = mbar_wait(&k_full[st], (uint32_t)(t / S) & 1u, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        v_left = (v_left & ~(3u << (2 * st))) | ((uint32_t)__popc(nw) << (2 * st));
+        if (nw == 0) tc_commit(&v_empty[st]);  // no warpgroup reads this tile's V
+        const uint32_t kbase = sKa + st * C::TILE;
+        if (nw & 1) ok = do_qk(0, t, kbase);
+        if (ok && (nw & 2)) ok = do_qk(1, t, kbase);
+        if (ok) tc_commit(&k_empty[st]);
+      }
+      if (ok && pend0 >= 0) ok = do_pv(0);
+      if (ok && pend1 >= 0) ok = do_pv(1);
+      if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax warpgroups
+    const int w = (warp - 2) >> 2;
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;              // row within the warpgroup's tile
+    const int pq = row0 + 128 * w + r;         // query position
+    const bool row_valid = pq < p.N;
+    const int grp = 2 * w + (r >> 6);
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t stm = tmem + lane_off + w * 128;
+    const uint32_t otm = tmem + lane_off + 256 + w * D;
+    const int Iq = (row_valid ? pq : (p.N - 1)) / p.block_q;
+    const size_t bias_row = ((size_t)h * p.nQB + Iq) * p.nKB;
+    const int my_bit = 1 << (kGrpShift + grp);
+
+    const QWin qw = gna_query_window(p.g, pq, p.has_gna && mode == BSA_HEAD_SPARSE);
+
+    const float cscale = p.scale_log2;
+    float m = kNegInf, l = 0.f;
+    int j = 0;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      if (!((tile_need(sched, nseg, t, act) >> w) & 1)) continue;
+      ok = warp_all(mbar_wait(&s_full[w], (uint32_t)j & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      const int ea = sched[2 * t];
+      const int eb = (2 * t + 1 < nseg) ? sched[2 * t + 1] : -1;
+      const int sa = ea & kSegIdxMask;
+      const int sb = eb >= 0 ? (eb & kSegIdxMask) : sa;
+      float ba = 0.f, bb = 0.f;
+      if (p.bias != nullptr) {
+        ba = __ldg(p.bias + bias_row + (sa * 64) / p.block_k) * kLog2e;
+        bb = __ldg(p.bias + bias_row + (sb * 64) / p.block_k) * kLog2e;
+      }
+      const bool tail = (sb + 1) * 64 > p.N || (sa + 1) * 64 > p.N;
+      const bool need = !(ea & my_bit) || eb < 0 || !(eb & my_bit) || tail ||
+                        ((ea | (eb < 0 ? 0 : eb)) & kPart4);
+      uint64_t ma = ~0ull, mb = ~0ull;
+      if (need) {
+        ma = 0ull;
+        mb = 0ull;
+        if (ea & my_bit) {
+          ma = tail_bits(p.N, sa);
+          if ((ea & kPart4) && p.has_gna) ma &= gna_segment_bits(p.g, sa, qw);
+        }
+        if (eb >= 0 && (eb & my_bit)) {
+          mb = tail_bits(p.N, sb);
+          if ((eb & kPart4) && p.has_gna) mb &= gna_segment_bits(p.g, sb, qw);
+        }
+      }
+      // pass 1: row max of the raw scores, per 64-key half (the bias is constant per half)
+      float xa, xb;
+      {
+        float r[64];
+        tmem_ld32(stm, r);
+        tmem_ld32(stm + 32, r + 32);
+        tc_wait_ld();
+        if (need) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) r[i] = ((ma >> i) & 1ull) ? r[i] : kNegInf;
+        }
+        xa = max3f(r[0], r[1], r[2]);
+#pragma unroll
+        for (int i = 3; i < 63; i += 2) xa = max3f(xa, r[i], r[i + 1]);
+        xa = fmaxf(xa, r[63]);
+        tmem_ld32(stm + 64, r);
+        tmem_ld32(stm + 96, r + 32);
+        tc_wait_ld();
+        if (need) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) r[i] = ((mb >> i) & 1ull) ? r[i] : kNegInf;
+        }
+        xb = max3f(r[0], r[1], r[2]);
+#pragma unroll
+        for (int i = 3; i < 63; i += 2) xb = max3f(xb, r[i], r[i + 1]);
+        xb = fmaxf(xb, r[63]);
+      }
+      const float ta = (xa == kNegInf) ? kNegInf : fmaf(xa, cscale, ba);
+      const float tb = (xb == kNegInf) ? kNegInf : fmaf(xb, cscale, bb);
+      const float m_new = max3f(m, ta, tb);
+      float alpha = 1.f;
+      if (m_new > m + kRescaleTau) {
+        alpha = fast_exp2(m - m_new);
+        m = m_new;
+      }
+      const float mu = (m == kNegInf) ? 0.f : m;
+      const float oa = ba - mu, ob = bb - mu;
+      // pass 2: P = exp2(x - m) per 32-key chunk, packed to bf16 over the scores
+      // (chunk c's P lands in columns [16c, 16c + 16), all already read)
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float r[32];
+        tmem_ld32(stm + 32 * c, r);
+        tc_wait_ld();
+        if (need) {
+          const uint32_t bits = (uint32_t)((c < 2 ? ma : mb) >> (32 * (c & 1)));
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = ((bits >> i) & 1u) ? r[i] : kNegInf;
+        }
+        const float o = c < 2 ? oa : ob;
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0 = r[2 * i], x1 = r[2 * i + 1];
+          fma2(x0, x1, cscale, o);
+          if ((i & 7) < kEmuPairsPer8) {
+            poly_exp2_2(x0, x1);
+          } else {
+            x0 = fast_exp2(x0);
+            x1 = fast_exp2(x1);
+          }
+          add2(sum0, sum1, x0, x1);
+          pk[i] = pack_bf16x2(x0, x1);
+        }
+        tmem_st16(stm + 16 * c, pk);
+      }
+      l = l * alpha + (sum0 + sum1);
+      if (j > 0) {
+        ok = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(otm + c * 32, o);
+            tc_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(otm + c * 32, reinterpret_cast<uint32_t*>(o));
+          }
+        }
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[w]);
+      ++j;
+    }
+    if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+
+    // ---------------------------------------------------------------- epilogue
+    bool have = ok && j > 0;
+    if (have) {
+      have = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
+      if (!have) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+      tc_fence_after();
+    }
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    uint8_t* stage = sQ + w * C::TILE;  // the Q tile is no longer read once O is final
+    const size_t obase = ((size_t)bh * p.N + (row_valid ? pq : 0)) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      if (have) {
+        tmem_ld32(otm + c * 32, o);
+        tc_wait_ld();
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] *= inv;
+      const int chunk = c >> 1;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 v;
+        v.x = pack_bf16x2(o[8 * q + 0], o[8 * q + 1]);
+        v.y = pack_bf16x2(o[8 * q + 2], o[8 * q + 3]);
+        v.z = pack_bf16x2(o[8 * q + 4], o[8 * q + 5]);
+        v.w = pack_bf16x2(o[8 * q + 6], o[8 * q + 7]);
+        const int unit = 4 * (c & 1) + q;
+        *reinterpret_cast<uint4*>(stage + chunk * C::CHUNK + r * 128 + ((unit ^ (r & 7)) << 4)) = v;
+      }
+      if (p.cache_out != nullptr && row_valid) {
+        float4* cd = reinterpret_cast<float4*>(p.cache_out + obase + c * 32);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) cd[q] = make_float4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar(1 + w, 128);
+    if (q4 == 0 && lane == 0 && (act >> w) & 1) {
+      for (int c = 0; c < D / 64; ++c)
+        for (int rr = 0; rr < 2; ++rr)
+          if (row0 + 128 * w + 64 * rr < p.N)
+            tma_store_3d(&tmO, stage + c * C::CHUNK + rr * (C::CHUNK / 2), c * 64, row0 + 128 * w + 64 * rr,
+                         bh);
+      bulk_commit();
+      bulk_wait_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+static cudaError_t launch_fwd_d(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                                const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
+  auto fn = fwd_kernel<D>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  fn<<<grid, 320, FwdCfg<D>::SMEM_ALLOC, stream>>>(q, k, v, o, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_forward(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                           const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
+  if (d == 64) return launch_fwd_d<64>(q, k, v, o, p, grid, stream);
+  return launch_fwd_d<128>(q, k, v, o, p, grid, stream);
+}
+
+}  // namespace bsa

@@ -1,0 +1,252 @@
+// The two score passes of the SparseD full-score selection ("Isolated
+// Selection": A = attention map, A' = avgpool(A, block_size), top-rho% per
+// query block and key group), on tcgen05 tensor cores.
+//
+//   KIND_LSE   per-row log-sum-exp (log2 units) of scale*q.k + bias over all keys
+//   KIND_POOL  given the LSE, the block sums of softmax(z), i.e. the numerators
+//              of A'[I, J]; every 128-row query tile adds its 128 rows into
+//              A'[I, J] (one atomic per warp and 64-key half)
+//
+// One CTA computes one 128-row query tile of one (b, h) against every key.
+// Roles (192 threads): warp 0 TMA producer (Q once, K tiles into a ring),
+// warp 1 TMEM allocator and single-thread tcgen05.mma issuer (S = Q K^T into
+// a double-buffered fp32 accumulator in tensor memory), warps 2-5 one thread
+// per row reading S from tensor memory.
+#include "tiles.cuh"
+
+namespace bsa {
+
+template <int D>
+struct ScoreCfg {
+  static constexpr int STAGES = D == 64 ? 4 : 3;
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int CHUNK_BYTES = 128 * 128;
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = TILE_BYTES;
+  static constexpr int BAR_OFF = K_OFF + STAGES * TILE_BYTES;
+  static constexpr int NBAR = 1 + 2 * STAGES + 4;  // q_full, k_full[S], k_empty[S], s_full[2], s_free[2]
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 64;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+};
+static_assert(ScoreCfg<128>::SMEM_ALLOC <= 227 * 1024, "smem budget");
+
+template <int D, int KIND>
+__global__ void __launch_bounds__(192, 1)
+    score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const AttnParams p) {
+  using C = ScoreCfg<D>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qt = blockIdx.x % p.nQT;
+  const int bh = blockIdx.x / p.nQT;
+  const int h = bh % p.H;
+  const int row0 = qt * 128;
+  const int T = (p.N + 127) >> 7;  // 128-key tiles
+
+  uint8_t* sQ = smem + C::Q_OFF;
+  uint8_t* sK = smem + C::K_OFF;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* k_empty = k_full + S;
+  uint64_t* s_full = k_empty + S;
+  uint64_t* s_free = s_full + 2;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_free[b], 128);
+    }
+    misc[1] = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(misc, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
+      for (int c = 0; c < D / 64; ++c)
+        for (int r = 0; r < 2; ++r)
+          tma_load_3d(sQ + c * C::CHUNK_BYTES + r * (C::CHUNK_BYTES / 2), &tmQ, q_full, c * 64, row0 + 64 * r, bh);
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % S;
+        if (t >= S && !mbar_wait(&k_empty[st], ((uint32_t)(t / S) & 1u) ^ 1u, abort_flag)) {
+          cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(&k_full[st], C::TILE_BYTES);
+        uint8_t* dk = sK + st * C::TILE_BYTES;
+        for (int c = 0; c < D / 64; ++c)
+          for (int r = 0; r < 2; ++r)
+            tma_load_3d(dk + c * C::CHUNK_BYTES + r * (C::CHUNK_BYTES / 2), &tmK, &k_full[st], c * 64,
+                        t * 128 + 64 * r, bh);
+        issued = t + 1;
+      }
+      if (*abort_flag) {
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(smem_u32(q_full), 0u) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
+        for (int t = issued - S < 0 ? 0 : issued - S; t < issued; ++t)
+          while (!mbar_try_wait(smem_u32(&k_full[t % S]), (uint32_t)(t / S) & 1u) &&
+                 globaltimer_ns() - t0 < kWaitLimitNs) {
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
+      bool ok = mbar_wait(q_full, 0u, abort_flag);
+      for (int t = 0; t < T && ok; ++t) {
+        const int st = t % S, buf = t & 1;
+        if (t >= 2) ok = mbar_wait(&s_free[buf], (uint32_t)((t - 2) >> 1) & 1u, abort_flag);
+        ok = ok && mbar_wait(&k_full[st], (uint32_t)(t / S) & 1u, abort_flag);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t kbase = sKa + st * C::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          umma_ss(tmem + buf * 128, smem_desc_sw128(sQa + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
+                  idesc, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&s_full[buf]);
+        tc_commit(&k_empty[st]);
+      }
+      if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+    }
+  } else {
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const int pq = row0 + r;
+    const bool row_valid = pq < p.N;
+    const uint32_t lbase = tmem + ((uint32_t)(q4 * 32) << 16);
+    const int Iq = (row_valid ? pq : (p.N - 1)) / p.block_q;
+    const size_t bias_row = ((size_t)h * p.nQB + Iq) * p.nKB;
+    float m = kNegInf, l = 0.f;
+    const float lse2 = (KIND == KIND_POOL && row_valid) ? p.lse[(size_t)bh * p.N + pq] : 0.f;
+    bool ok = true;
+    float s[128];
+    for (int t = 0; t < T; ++t) {
+      const int buf = t & 1;
+      ok = warp_all(mbar_wait(&s_full[buf], (uint32_t)(t >> 1) & 1u, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lbase + buf * 128 + c * 32, s + c * 32);
+      tc_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&s_free[buf]);
+      const int sa = 2 * t, sb = 2 * t + 1;  // 64-key halves of the tile
+      float ba = 0.f, bb = 0.f;
+      if (p.bias != nullptr) {
+        ba = __ldg(p.bias + bias_row + (sa * 64) / p.block_k) * kLog2e;
+        if (sb < p.nSeg) bb = __ldg(p.bias + bias_row + (sb * 64) / p.block_k) * kLog2e;
+      }
+#pragma unroll
+      for (int j = 0; j < 64; ++j) s[j] = fmaf(s[j], p.scale_log2, ba);
+#pragma unroll
+      for (int j = 64; j < 128; ++j) s[j] = fmaf(s[j], p.scale_log2, bb);
+      if ((t + 1) * 128 > p.N) {  // ragged last tile: keys past N do not exist
+        const uint64_t ma = tail_bits(p.N, sa);
+        const uint64_t mb = sb < p.nSeg ? tail_bits(p.N, sb) : 0ull;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) s[j] = ((ma >> j) & 1ull) ? s[j] : kNegInf;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) s[64 + j] = ((mb >> j) & 1ull) ? s[64 + j] : kNegInf;
+      }
+      if (KIND == KIND_LSE) {
+        float mx = s[0];
+#pragma unroll
+        for (int j = 1; j < 128; ++j) mx = fmaxf(mx, s[j]);
+        const float m_new = fmaxf(m, mx);
+        if (m_new > m) {
+          l *= fast_exp2(m - m_new);
+          m = m_new;
+        }
+        const float mu = (m == kNegInf) ? 0.f : m;
+        float sum = 0.f;
+#pragma unroll
+        for (int j = 0; j < 128; ++j) sum += fast_exp2(s[j] - mu);
+        l += sum;
+      } else {
+        float suma = 0.f, sumb = 0.f;
+#pragma unroll
+        for (int j = 0; j < 64; ++j) suma += fast_exp2(s[j] - lse2);
+#pragma unroll
+        for (int j = 64; j < 128; ++j) sumb += fast_exp2(s[j] - lse2);
+        if (!row_valid) suma = sumb = 0.f;
+        const int Ja = (sa * 64) / p.block_k, Jb = (sb * 64) / p.block_k;
+        if (Ja == Jb) {
+          suma += sumb;
+          sumb = 0.f;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          suma += __shfl_xor_sync(0xffffffffu, suma, o);
+          sumb += __shfl_xor_sync(0xffffffffu, sumb, o);
+        }
+        if (lane == 0) {
+          float* dst = p.apool + ((size_t)bh * p.nQB + Iq) * p.nKB;
+          atomicAdd(dst + Ja, suma);
+          if (Ja != Jb && sb < p.nSeg) atomicAdd(dst + Jb, sumb);
+        }
+      }
+    }
+    if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+    if (KIND == KIND_LSE && row_valid) p.lse[(size_t)bh * p.N + pq] = (l > 0.f) ? m + __log2f(l) : kNegInf;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+template <int D, int KIND>
+static cudaError_t launch_score_d(const CUtensorMap& q, const CUtensorMap& k, const AttnParams& p, int grid,
+                                  cudaStream_t stream) {
+  auto fn = score_kernel<D, KIND>;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreCfg<D>::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  fn<<<grid, 192, ScoreCfg<D>::SMEM_ALLOC, stream>>>(q, k, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_score(int d, int kind, const CUtensorMap& q, const CUtensorMap& k, const AttnParams& p,
+                         int grid, cudaStream_t stream) {
+  if (d == 64)
+    return kind == KIND_LSE ? launch_score_d<64, KIND_LSE>(q, k, p, grid, stream)
+                            : launch_score_d<64, KIND_POOL>(q, k, p, grid, stream);
+  return kind == KIND_LSE ? launch_score_d<128, KIND_LSE>(q, k, p, grid, stream)
+                          : launch_score_d<128, KIND_POOL>(q, k, p, grid, stream);
+}
+
+}  // namespace bsa

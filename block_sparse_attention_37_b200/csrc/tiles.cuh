@@ -1,0 +1,117 @@
+// Helpers for 64-key segments and the GNA fine mask, shared by the forward
+// and the selection score passes.
+#pragma once
+
+#include "attention.cuh"
+
+namespace bsa {
+
+#define kNegInf (-__int_as_float(0x7f800000))
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kSegIdxMask = (1 << 24) - 1;
+
+__device__ __forceinline__ void cta_fail(volatile int* abort_flag, int code) {
+  *abort_flag = 1;
+  record_error(code);
+}
+
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+__device__ __forceinline__ uint32_t bit_range(int a, int b) {  // bits [a, b), clipped to [0, 32)
+  a = max(a, 0);
+  b = min(b, 32);
+  if (a >= b) return 0u;
+  const uint32_t hi = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  const uint32_t lo = (1u << a) - 1u;
+  return hi & ~lo;
+}
+
+__device__ __forceinline__ uint64_t bit_range64(int a, int b) {  // bits [a, b), clipped to [0, 64)
+  a = max(a, 0);
+  b = min(b, 64);
+  if (a >= b) return 0ull;
+  const uint64_t hi = b >= 64 ? ~0ull : ((1ull << b) - 1ull);
+  const uint64_t lo = (1ull << a) - 1ull;
+  return hi & ~lo;
+}
+
+// Keys of segment `seg` below N.
+__device__ __forceinline__ uint64_t tail_bits(int N, int seg) {
+  const int n = N - seg * 64;
+  return n >= 64 ? ~0ull : ((1ull << n) - 1ull);
+}
+
+// Does KV block J of a GNA tile layout hold padded (invalid) key slots?
+__device__ __forceinline__ bool gna_block_padded(const GnaDev& g, int J) {
+  const int ntb = g.text_span / g.vol;
+  if (J < ntb) return g.text_span > g.n_text && (J + 1) * g.vol > g.n_text;
+  const int tile = J - ntb;
+  const int c2 = tile % g.tiles[2];
+  const int c1 = (tile / g.tiles[2]) % g.tiles[1];
+  const int c0 = tile / (g.tiles[2] * g.tiles[1]);
+  return (c0 + 1) * g.tile[0] > g.grid[0] || (c1 + 1) * g.tile[1] > g.grid[1] ||
+         (c2 + 1) * g.tile[2] > g.grid[2];
+}
+
+// A query's key window per dimension, [lo, hi) (text and full rows: everything).
+struct QWin {
+  int lo0, lo1, lo2, hi0, hi1, hi2;
+};
+
+__device__ __forceinline__ QWin gna_query_window(const GnaDev& g, int pq, bool windowed) {
+  QWin w{0, 0, 0, 1 << 30, 1 << 30, 1 << 30};
+  if (!windowed || pq < g.text_span) return w;
+  const int v = pq - g.text_span;
+  const int tile = v / g.vol, l = v - tile * g.vol;
+  const int c0 = (tile / (g.tiles[2] * g.tiles[1])) * g.tile[0] + l / (g.tile[1] * g.tile[2]);
+  const int c1 = ((tile / g.tiles[2]) % g.tiles[1]) * g.tile[1] + (l / g.tile[2]) % g.tile[1];
+  const int c2 = (tile % g.tiles[2]) * g.tile[2] + l % g.tile[2];
+  if (c0 >= g.grid[0] || c1 >= g.grid[1] || c2 >= g.grid[2]) return w;  // padding row
+  w.lo0 = gna_window_start(c0, g.grid[0], g.win[0], g.stride[0]);
+  w.lo1 = gna_window_start(c1, g.grid[1], g.win[1], g.stride[1]);
+  w.lo2 = gna_window_start(c2, g.grid[2], g.win[2], g.stride[2]);
+  w.hi0 = w.lo0 + g.win[0];
+  w.hi1 = w.lo1 + g.win[1];
+  w.hi2 = w.lo2 + g.win[2];
+  return w;
+}
+
+// Allowed-key bits of one 64-key segment (tile order) for a query window.
+// Needs the tile's x-extent to divide 64 or be a multiple of 64.
+__device__ __forceinline__ uint64_t gna_segment_bits(const GnaDev& g, int seg, const QWin& q) {
+  const int k0 = seg * 64;
+  if (k0 < g.text_span) {
+    const int nt = g.n_text - k0;
+    return nt <= 0 ? 0ull : (nt >= 64 ? ~0ull : ((1ull << nt) - 1ull));
+  }
+  const int v0 = k0 - g.text_span;
+  const int tile = v0 / g.vol;
+  const int l0 = v0 - tile * g.vol;
+  const int tx = tile % g.tiles[2];
+  const int ty = (tile / g.tiles[2]) % g.tiles[1];
+  const int tt = tile / (g.tiles[2] * g.tiles[1]);
+  const int bt = tt * g.tile[0], by = ty * g.tile[1], bx = tx * g.tile[2];
+  const int Tx = g.tile[2], Ty = g.tile[1];
+  const int xlo = max(q.lo2, 0), xhi = min(q.hi2, g.grid[2]);
+  uint64_t m = 0ull;
+  if (Tx <= 64) {
+    const int rows = 64 / Tx;
+    const int R0 = l0 / Tx;
+    const uint64_t xb = bit_range64(xlo - bx, xhi - bx) & bit_range64(0, Tx);
+    for (int rr = 0; rr < rows; ++rr) {
+      const int R = R0 + rr;
+      const int t = bt + R / Ty, y = by + R % Ty;
+      const bool ok = t >= q.lo0 && t < q.hi0 && t < g.grid[0] && y >= q.lo1 && y < q.hi1 && y < g.grid[1];
+      if (ok) m |= xb << (rr * Tx);
+    }
+  } else {
+    const int R = l0 / Tx;
+    const int xo = bx + (l0 - R * Tx);
+    const int t = bt + R / Ty, y = by + R % Ty;
+    const bool ok = t >= q.lo0 && t < q.hi0 && t < g.grid[0] && y >= q.lo1 && y < q.hi1 && y < g.grid[1];
+    if (ok) m = bit_range64(xlo - xo, xhi - xo);
+  }
+  return m;
+}
+
+}  // namespace bsa
