@@ -147,7 +147,7 @@ def _bsa():
 def source_sha():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "block_sparse_attention_37_b200", "csrc")
-    for f in ("attention.cu", "attention.cuh", "common.cuh"):
+    for f in ("forward.cu", "tiles.cuh", "attention.cuh", "common.cuh"):
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -535,7 +535,7 @@ def run_bsa(args, rank, world, local_rank):
     key = f"attn_fwd_{cfg}"
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic_for(key),
-            "kernel": "bsa::attn_kernel<D,KIND_FWD> (bsa_forward)",
+            "kernel": "bsa::fwd_kernel<D> (bsa_forward)",
             "peak_source": f"{peak_src} bf16 burst (kernel timed alone between L2 flushes)",
             "algorithmic_flops_per_launch": job.flops}
     line = {

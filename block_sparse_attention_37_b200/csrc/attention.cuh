@@ -27,7 +27,6 @@ struct AttnParams {
   __nv_bfloat16* O;          // [B,H,N,d]
   float* lse;                // [B,H,N] log2-domain row LSE (LSE out, POOL in)
   float* apool;              // [B,H,nQB,nKB] block sums of softmax (POOL out)
-  const int32_t* order;      // optional CTA -> work item permutation
   int has_gna;
   GnaDev g;
 };

@@ -5,17 +5,22 @@
 // kept 64-key segments, with one validity bit per group; a warpgroup skips a
 // 128-key tile none of its rows keeps, so each tile costs tensor work only
 // for the warpgroups that need it while K and V are loaded once.
-// Roles (320 threads):
-//   warp 0     TMA producer: both Q tiles, then K/V tiles into a shared ring
-//   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2-5  softmax warpgroup 0 (rows 0..127 of the CTA)
-//   warps 6-9  softmax warpgroup 1 (rows 128..255)
+// Roles (384 threads, three aligned warpgroups):
+//   warp 0      TMA producer: both Q tiles, then K/V tiles into a shared ring
+//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 2-3   idle (they complete the control warpgroup)
+//   warps 4-7   softmax warpgroup 0 (rows 0..127 of the CTA)
+//   warps 8-11  softmax warpgroup 1 (rows 128..255)
+// The control warpgroup hands registers to the softmax warpgroups
+// (setmaxnreg), which keep a whole 128-key row of S in registers.
 // Tensor memory (512 columns): S/P of warpgroup w at column 128w, O of
 // warpgroup w at 256 + w*D. The MMA warp alternates the two warpgroups, so
 // the tensor core runs one group's PV and next QK^T while the other group's
 // softmax runs (lmnt.cn BSA post, section 3.1: FlashAttention tiles with
 // online softmax over the selected blocks; DiTFastAttnV2 "Fused Kernel").
 // Output leaves through shared memory and a TMA store.
+#include <utility>
+
 #include "tiles.cuh"
 
 namespace bsa {
@@ -31,19 +36,47 @@ struct FwdCfg {
   static constexpr int K_OFF = 2 * TILE;
   static constexpr int V_OFF = K_OFF + STAGES * TILE;
   static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
-  static constexpr int NBAR = 2 + 4 * STAGES + 6;
+  static constexpr int NBAR = 2 + 6 * STAGES + 8;
+  // d = 64: P gets its own tensor-memory columns (S 128 + P 64 + O 64 per
+  // warpgroup fill all 512), so the next QK^T can overwrite S as soon as the
+  // softmax has read it; d = 128: P is written over S and waits for PV.
+  static constexpr bool SEP_P = D == 64;
+  static constexpr uint32_t S_COL = 0;                     // + 128 w
+  static constexpr uint32_t P_COL = SEP_P ? 256 : 0;       // + (SEP_P ? 64 : 128) w
+  static constexpr uint32_t P_STRIDE = SEP_P ? 64 : 128;
+  static constexpr uint32_t O_COL = SEP_P ? 384 : 256;     // + D w
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BITS_OFF = MISC_OFF + 64;
   static constexpr int SCHED_OFF = BITS_OFF + 5 * 64 * 4;
   static constexpr int SMEM_BYTES = SCHED_OFF + kMaxSeg * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+  // register split: launched at kLaunchRegs per thread, the control
+  // warpgroup drops to REGS_CTL and the two softmax warpgroups rise to REGS_SMX
+  static constexpr int THREADS = 384;
+  static constexpr int REGS_CTL = 56;
+  static constexpr int REGS_SMX = 224;
 };
+constexpr int kLaunchRegs = 168;  // 65536 / 384, rounded down to a multiple of 8
+template <int D>
+constexpr bool regs_fit() {
+  return 128 * FwdCfg<D>::REGS_CTL + 256 * FwdCfg<D>::REGS_SMX <= FwdCfg<D>::THREADS * kLaunchRegs;
+}
+static_assert(regs_fit<64>() && regs_fit<128>(), "register split exceeds the launch allocation");
 static_assert(FwdCfg<128>::SMEM_ALLOC <= 227 * 1024, "smem budget");
 static_assert(FwdCfg<64>::SMEM_ALLOC <= 227 * 1024, "smem budget");
 
 // Segment entry bits: index in [0, 24), group-valid bits g0..g3 at 24..27, partial at 28.
 constexpr int kGrpShift = 24;
 constexpr int kPart4 = 1 << 28;
+
+template <int N>
+__device__ __forceinline__ void regs_release() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_claim() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
 
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -123,8 +156,12 @@ __device__ __forceinline__ void poly_exp2_2(float& x0, float& x1) {
   x1 = __int_as_float(max((int)p1, 0));
 }
 
-// Of every 8 exponent pairs of a row, how many go to the FMA pipe.
-constexpr int kEmuPairsPer8 = 2;
+// Of every 8 exponent pairs of a row, how many go to the FMA pipe (measured:
+// helps at d = 64 where the softmax dominates, costs at d = 128).
+template <int D>
+__host__ __device__ constexpr int emu_pairs_per8() {
+  return D == 64 ? 2 : 0;
+}
 
 // Fill one group's segment bits from a block-list row.
 __device__ void fill_group_bits(const AttnParams& p, size_t row, uint32_t* vb, uint32_t* pb, int lane) {
@@ -247,6 +284,32 @@ __device__ __forceinline__ int tile_need(const int32_t* sched, int nseg, int t, 
   return (((g & 3) ? 1 : 0) | ((g & 12) ? 2 : 0)) & act_mask;
 }
 
+// S = Q K^T over D/16 k-steps of 16 (K-major SW128 operands: k-step kk sits
+// in 64-column chunk kk/4 (16 KB apart) at byte offset 32*(kk%4)).
+template <int KK>
+__device__ __forceinline__ void qk_step(uint32_t s_tmem, uint64_t qd, uint64_t kd, uint32_t idesc) {
+  constexpr uint32_t off = ((KK >> 2) * 16384 + (KK & 3) * 32) >> 4;
+  umma_ss_at_warp<off, off>(s_tmem, qd, kd, idesc, KK > 0 ? 1u : 0u);
+}
+template <int... KK>
+__device__ __forceinline__ void qk_all(uint32_t s_tmem, uint64_t qd, uint64_t kd, uint32_t idesc,
+                                       std::integer_sequence<int, KK...>) {
+  (qk_step<KK>(s_tmem, qd, kd, idesc), ...);
+}
+
+// O (+)= P V over 8 k-steps of 16 keys: P from tensor memory (8 columns per
+// step), V MN-major SW128 (16 rows = 2048 bytes per step).
+template <int KK>
+__device__ __forceinline__ void pv_step(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd, uint32_t idesc, uint32_t first) {
+  constexpr uint32_t voff = KK * 2048 / 16;
+  umma_ts_at_warp<KK * 8, voff>(o_tmem, p_tmem, vd, idesc, (KK > 0 || !first) ? 1u : 0u);
+}
+template <int... KK>
+__device__ __forceinline__ void pv_all(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd, uint32_t idesc, uint32_t first,
+                                       std::integer_sequence<int, KK...>) {
+  (pv_step<KK>(o_tmem, p_tmem, vd, idesc, first), ...);
+}
+
 template <int D>
 __device__ void skip_copy256(const AttnParams& p, int bh, int row0) {
   if (p.cache_in == nullptr) {
@@ -268,7 +331,7 @@ __device__ void skip_copy256(const AttnParams& p, int bh, int row0) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                const AttnParams p) {
@@ -279,9 +342,8 @@ __global__ void __launch_bounds__(320, 1)
                                              ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nQP = (p.N + 255) >> 8;
-  const int work = p.order ? p.order[blockIdx.x] : (int)blockIdx.x;
-  const int pair = work % nQP;
-  const int bh = work / nQP;
+  const int pair = (int)blockIdx.x % nQP;
+  const int bh = (int)blockIdx.x / nQP;
   const int h = bh % p.H;
   const int row0 = pair * 256;
 
@@ -301,12 +363,13 @@ __global__ void __launch_bounds__(320, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::BAR_OFF);
   uint64_t* q_full = bars;          // [2]
   uint64_t* k_full = bars + 2;      // [S]
-  uint64_t* k_empty = k_full + S;   // [S]
-  uint64_t* v_full = k_empty + S;   // [S]
-  uint64_t* v_empty = v_full + S;   // [S]
-  uint64_t* s_full = v_empty + S;   // [2]
+  uint64_t* v_full = k_full + S;         // [S]
+  uint64_t* k_empty = v_full + S;        // [S][2]: stage released by warpgroup w
+  uint64_t* v_empty = k_empty + 2 * S;   // [S][2]
+  uint64_t* s_full = v_empty + 2 * S;  // [2]
   uint64_t* p_full = s_full + 2;    // [2]
   uint64_t* o_ready = p_full + 2;   // [2]
+  uint64_t* s_free = o_ready + 2;   // [2] (separate-P layout: S read by the softmax)
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   uint32_t* vb = reinterpret_cast<uint32_t*>(smem + C::BITS_OFF);
@@ -318,11 +381,14 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(&s_full[w], 1);
       mbar_init(&p_full[w], 128);
       mbar_init(&o_ready[w], 1);
+      mbar_init(&s_free[w], 128);
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
       mbar_init(&v_full[s], 1);
+    }
+    for (int s = 0; s < 2 * S; ++s) {
+      mbar_init(&k_empty[s], 1);
       mbar_init(&v_empty[s], 1);
     }
     misc[1] = 0;
@@ -364,7 +430,19 @@ __global__ void __launch_bounds__(320, 1)
   const int act = (int)misc[5];
   const int wg_tiles0 = (int)misc[3], wg_tiles1 = (int)misc[4];
 
-  if (warp == 0) {
+  // every role ends with its own copy of the teardown (a shared tail would
+  // make the register allocator apply the control warpgroup's limit to all)
+  auto teardown = [&]() {
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+      tc_fence_after();
+      tmem_dealloc(tmem, 512);
+    }
+  };
+  if (warp < 4) {
+    regs_release<C::REGS_CTL>();
+    if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0 && T > 0) {
       tma_prefetch_desc(&tmQ);
@@ -380,12 +458,21 @@ __global__ void __launch_bounds__(320, 1)
                         row0 + 128 * w + 64 * r, bh);
       }
       int k_issued = 0, v_issued = 0;
+      uint32_t kpar = 0u, vpar = 0u;  // phase parity per (stage, warpgroup) release barrier
       for (int t = 0; t < T; ++t) {
         const int st = t % S;
-        const uint32_t ph = (uint32_t)(t / S) & 1u;
         const int sa = sched[2 * t] & kSegIdxMask;
         const int sb = (2 * t + 1 < nseg) ? (sched[2 * t + 1] & kSegIdxMask) : sa;
-        if (t >= S && !mbar_wait(&k_empty[st], ph ^ 1u, abort_flag)) {
+        // the warpgroups that used this stage's previous tile must have released it
+        const int prev_need = t >= S ? tile_need(sched, nseg, t - S, act) : 0;
+        bool released = true;
+        for (int w = 0; w < 2 && released; ++w)
+          if ((prev_need >> w) & 1) {
+            const int b = 2 * st + w;
+            released = mbar_wait(&k_empty[b], (kpar >> b) & 1u, abort_flag);
+            kpar ^= 1u << b;
+          }
+        if (!released) {
           cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
           break;
         }
@@ -396,7 +483,13 @@ __global__ void __launch_bounds__(320, 1)
           tma_load_3d(dk + c * C::CHUNK + C::CHUNK / 2, &tmK, &k_full[st], c * 64, sb * 64, bh);
         }
         k_issued = t + 1;
-        if (t >= S && !mbar_wait(&v_empty[st], ph ^ 1u, abort_flag)) {
+        for (int w = 0; w < 2 && released; ++w)
+          if ((prev_need >> w) & 1) {
+            const int b = 2 * st + w;
+            released = mbar_wait(&v_empty[b], (vpar >> b) & 1u, abort_flag);
+            vpar ^= 1u << b;
+          }
+        if (!released) {
           cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
           break;
         }
@@ -422,94 +515,128 @@ __global__ void __launch_bounds__(320, 1)
           drain(&v_full[t % S], (uint32_t)(t / S) & 1u);
       }
     }
-  } else if (warp == 1) {
+    } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    if (lane == 0 && T > 0) {
+    // The warp serves both warpgroups by polling: whichever QK^T or PV is
+    // ready is issued, so neither warpgroup waits behind the other's barriers.
+    // All 32 lanes run the loop, so its state and the operand descriptors are
+    // warp-uniform; one elected lane issues each MMA and commit.
+    if (T > 0) {
+      auto ready = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return __all_sync(0xffffffffu, mbar_test(smem_u32(bar), parity));
+      };
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      bool ok = true;
-      // per-warpgroup state in scalars (no local memory on the issue path)
-      int pend0 = -1, pend1 = -1;  // tile whose PV is still to be issued
-      int done0 = 0, done1 = 0;    // QK^T tiles issued
-      uint32_t q_ok = 0u;          // bit w: Q tile w has landed
-      uint32_t v_left = 0u;        // 2 bits per stage: PVs still to read that stage's V
-      auto do_pv = [&](int w) -> bool {
-        const int u = w ? pend1 : pend0;
-        const int j = (w ? done1 : done0) - 1;
-        const int st = u % S;
-        if (!mbar_wait(&p_full[w], (uint32_t)j & 1u, abort_flag)) return false;
-        if (!mbar_wait(&v_full[st], (uint32_t)(u / S) & 1u, abort_flag)) return false;
+      // per-warpgroup state: next tile to QK (T = none), QK^T count, and the
+      // tiles whose PV is outstanding in issue order (f0 first), with their
+      // indices among the warpgroup's tiles
+      struct WgState {
+        int next, cnt, f0, j0, f1, j1;
+        bool q_ok;
+      };
+      auto next_tile = [&](int t, int w) {
+        while (t < T && !((tile_need(sched, nseg, t, act) >> w) & 1)) ++t;
+        return t;
+      };
+      WgState g0{next_tile(0, 0), 0, -1, 0, -1, 0, wg_tiles0 == 0};
+      WgState g1{next_tile(0, 1), 0, -1, 0, -1, 0, wg_tiles1 == 0};
+      // K and V tiles are observed landing in tile order: when tile x is
+      // tested, tile x - S (same stage) is known to have landed and tile
+      // x + S cannot have been loaded (its stage waits for the users of x),
+      // so a one-bit parity test cannot alias another phase of the stage
+      int k_seen = 0, v_seen = 0;
+      // PV of the oldest outstanding tile, if its P and V are ready
+      auto try_pv = [&](WgState& g, int w) -> bool {
+        if (g.f0 < 0) return false;
+        const int u = g.f0, st = u % S;
+        while (v_seen <= u && ready(&v_full[v_seen % S], (uint32_t)(v_seen / S) & 1u)) ++v_seen;
+        if (v_seen <= u || !ready(&p_full[w], (uint32_t)g.j0 & 1u)) return false;
         tc_fence_after();
-        const uint32_t vbase = sVa + st * C::TILE;
-        const uint32_t ptm = tmem + w * 128, otm = tmem + 256 + w * D;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(otm, ptm + kk * 8, smem_desc_sw128(vbase + kk * 2048, C::CHUNK, 1024), idesc_pv,
-                  (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(&o_ready[w]);
-        const uint32_t left = ((v_left >> (2 * st)) & 3u) - 1u;
-        v_left = (v_left & ~(3u << (2 * st))) | (left << (2 * st));
-        if (left == 0) tc_commit(&v_empty[st]);
-        if (w) pend1 = -1; else pend0 = -1;
+        pv_all(tmem + C::O_COL + w * D, tmem + C::P_COL + w * C::P_STRIDE,
+               smem_desc_sw128(sVa + st * C::TILE, C::CHUNK, 1024), idesc_pv, g.j0 == 0 ? 1u : 0u,
+               std::make_integer_sequence<int, 8>{});
+        tc_commit_warp(&o_ready[w]);
+        tc_commit_warp(&v_empty[2 * st + w]);
+        g.f0 = g.f1;
+        g.j0 = g.j1;
+        g.f1 = -1;
         return true;
       };
-      auto do_qk = [&](int w, int t, uint32_t kbase) -> bool {
-        if (!((q_ok >> w) & 1u)) {
-          if (!mbar_wait(&q_full[w], 0u, abort_flag)) return false;
-          tc_fence_after();
-          q_ok |= 1u << w;
+      // QK^T of the warpgroup's next tile, if Q, K and the S columns are ready
+      auto try_qk = [&](WgState& g, int w) -> bool {
+        if (g.next >= T || g.f1 >= 0) return false;
+        const int t = g.next, st = t % S;
+        if (!g.q_ok) {
+          if (!ready(&q_full[w], 0u)) return false;
+          g.q_ok = true;
         }
-        if ((w ? pend1 : pend0) >= 0 && !do_pv(w)) return false;
-        const uint32_t qbase = sQa + w * C::TILE;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-          umma_ss(tmem + w * 128, smem_desc_sw128(qbase + off, 16, 1024), smem_desc_sw128(kbase + off, 16, 1024),
-                  idesc_qk, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&s_full[w]);
-        if (w) {
-          pend1 = t;
-          ++done1;
+        // S is free once the softmax has read it (own P columns) or once the
+        // previous PV is issued (P written over S: the tensor pipe keeps order)
+        const bool s_ok = C::SEP_P ? (g.cnt == 0 || ready(&s_free[w], (uint32_t)(g.cnt - 1) & 1u))
+                                   : (g.f0 < 0);
+        if (!s_ok) return false;
+        while (k_seen <= t && ready(&k_full[k_seen % S], (uint32_t)(k_seen / S) & 1u)) ++k_seen;
+        if (k_seen <= t) return false;
+        tc_fence_after();
+        qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::TILE, 16, 1024),
+               smem_desc_sw128(sKa + st * C::TILE, 16, 1024), idesc_qk, std::make_integer_sequence<int, D / 16>{});
+        tc_commit_warp(&s_full[w]);
+        tc_commit_warp(&k_empty[2 * st + w]);
+        if (g.f0 < 0) {
+          g.f0 = t;
+          g.j0 = g.cnt;
         } else {
-          pend0 = t;
-          ++done0;
+          g.f1 = t;
+          g.j1 = g.cnt;
         }
+        ++g.cnt;
+        g.next = next_tile(t + 1, w);
         return true;
       };
-      for (int t = 0; t < T && ok; ++t) {
-        const int st = t % S;
-        // a PV still pending on this stage is issued before the stage is reused
-        if (pend0 >= 0 && pend0 % S == st) ok = do_pv(0);
-        if (ok && pend1 >= 0 && pend1 % S == st) ok = do_pv(1);
-        if (!ok) break;
-        const int nw = tile_need(sched, nseg, t, act);
-        ok = mbar_wait(&k_full[st], (uint32_t)(t / S) & 1u, abort_flag);
-        if (!ok) break;
-        tc_fence_after();
-        v_left = (v_left & ~(3u << (2 * st))) | ((uint32_t)__popc(nw) << (2 * st));
-        if (nw == 0) tc_commit(&v_empty[st]);  // no warpgroup reads this tile's V
-        const uint32_t kbase = sKa + st * C::TILE;
-        if (nw & 1) ok = do_qk(0, t, kbase);
-        if (ok && (nw & 2)) ok = do_qk(1, t, kbase);
-        if (ok) tc_commit(&k_empty[st]);
+      // separate P: the next QK^T first (it unblocks the softmax); shared columns: PV first
+      auto step = [&](WgState& g, int w) -> bool {
+        if (C::SEP_P) {
+          const bool q = try_qk(g, w);
+          return try_pv(g, w) || q;
+        }
+        const bool v = try_pv(g, w);
+        return try_qk(g, w) || v;
+      };
+      uint64_t t_idle = globaltimer_ns();
+      uint32_t spins = 0;
+      while (g0.next < T || g0.f0 >= 0 || g1.next < T || g1.f0 >= 0) {
+        const bool a0 = step(g0, 0);
+        const bool a1 = step(g1, 1);
+        if (a0 || a1) {
+          spins = 0;
+          continue;
+        }
+        if ((++spins & 63u) == 0) {
+          const uint64_t now = __shfl_sync(0xffffffffu, globaltimer_ns(), 0);
+          if (spins == 64) t_idle = now;
+          if (__any_sync(0xffffffffu, *abort_flag != 0) || now - t_idle > kWaitLimitNs) {
+            cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+            break;
+          }
+        }
       }
-      if (ok && pend0 >= 0) ok = do_pv(0);
-      if (ok && pend1 >= 0) ok = do_pv(1);
-      if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
     }
+    }
+    teardown();
   } else {
+    regs_claim<C::REGS_SMX>();
     // ---------------------------------------------------------------- softmax warpgroups
-    const int w = (warp - 2) >> 2;
+    const int w = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;              // row within the warpgroup's tile
     const int pq = row0 + 128 * w + r;         // query position
     const bool row_valid = pq < p.N;
     const int grp = 2 * w + (r >> 6);
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t stm = tmem + lane_off + w * 128;
-    const uint32_t otm = tmem + lane_off + 256 + w * D;
+    const uint32_t stm = tmem + lane_off + C::S_COL + w * 128;
+    const uint32_t ptm = tmem + lane_off + C::P_COL + w * C::P_STRIDE;
+    const uint32_t otm = tmem + lane_off + C::O_COL + w * D;
     const int Iq = (row_valid ? pq : (p.N - 1)) / p.block_q;
     const size_t bias_row = ((size_t)h * p.nQB + Iq) * p.nKB;
     const int my_bit = 1 << (kGrpShift + grp);
@@ -550,33 +677,34 @@ __global__ void __launch_bounds__(320, 1)
           if ((eb & kPart4) && p.has_gna) mb &= gna_segment_bits(p.g, sb, qw);
         }
       }
-      // pass 1: row max of the raw scores, per 64-key half (the bias is constant per half)
-      float xa, xb;
-      {
-        float r[64];
-        tmem_ld32(stm, r);
-        tmem_ld32(stm + 32, r + 32);
-        tc_wait_ld();
-        if (need) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) r[i] = ((ma >> i) & 1ull) ? r[i] : kNegInf;
-        }
-        xa = max3f(r[0], r[1], r[2]);
-#pragma unroll
-        for (int i = 3; i < 63; i += 2) xa = max3f(xa, r[i], r[i + 1]);
-        xa = fmaxf(xa, r[63]);
-        tmem_ld32(stm + 64, r);
-        tmem_ld32(stm + 96, r + 32);
-        tc_wait_ld();
-        if (need) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) r[i] = ((mb >> i) & 1ull) ? r[i] : kNegInf;
-        }
-        xb = max3f(r[0], r[1], r[2]);
-#pragma unroll
-        for (int i = 3; i < 63; i += 2) xb = max3f(xb, r[i], r[i + 1]);
-        xb = fmaxf(xb, r[63]);
+      // The whole 128-key row of S is read once into registers: with its own
+      // P columns, S is free for the next QK^T as soon as it has landed.
+      float sv[128];
+      tmem_ld32(stm, sv);
+      tmem_ld32(stm + 32, sv + 32);
+      tmem_ld32(stm + 64, sv + 64);
+      tmem_ld32(stm + 96, sv + 96);
+      tc_wait_ld();
+      if (C::SEP_P) {
+        tc_fence_before();
+        mbar_arrive(&s_free[w]);
       }
+      if (need) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) sv[i] = ((ma >> i) & 1ull) ? sv[i] : kNegInf;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) sv[64 + i] = ((mb >> i) & 1ull) ? sv[64 + i] : kNegInf;
+      }
+      // row max of the raw scores, per 64-key half (the bias is constant per half)
+      float xa = max3f(sv[0], sv[1], sv[2]);
+      float xb = max3f(sv[64], sv[65], sv[66]);
+#pragma unroll
+      for (int i = 3; i < 63; i += 2) {
+        xa = max3f(xa, sv[i], sv[i + 1]);
+        xb = max3f(xb, sv[64 + i], sv[65 + i]);
+      }
+      xa = fmaxf(xa, sv[63]);
+      xb = fmaxf(xb, sv[127]);
       const float ta = (xa == kNegInf) ? kNegInf : fmaf(xa, cscale, ba);
       const float tb = (xb == kNegInf) ? kNegInf : fmaf(xb, cscale, bb);
       const float m_new = max3f(m, ta, tb);
@@ -587,26 +715,26 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float mu = (m == kNegInf) ? 0.f : m;
       const float oa = ba - mu, ob = bb - mu;
-      // pass 2: P = exp2(x - m) per 32-key chunk, packed to bf16 over the scores
-      // (chunk c's P lands in columns [16c, 16c + 16), all already read)
+      // PV(j-1) must be complete before O is rescaled, and (own P columns)
+      // before P_w is overwritten; O is rescaled once S is dead (fewer live
+      // registers), which is safe because PV(j) waits for p_full
+      if (j > 0) {
+        ok = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      // P = exp2(x - m) per 32-key chunk, packed to bf16 (over the scores
+      // when P shares S's columns: S is already in registers)
       float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        float r[32];
-        tmem_ld32(stm + 32 * c, r);
-        tc_wait_ld();
-        if (need) {
-          const uint32_t bits = (uint32_t)((c < 2 ? ma : mb) >> (32 * (c & 1)));
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = ((bits >> i) & 1u) ? r[i] : kNegInf;
-        }
         const float o = c < 2 ? oa : ob;
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float x0 = r[2 * i], x1 = r[2 * i + 1];
+          float x0 = sv[32 * c + 2 * i], x1 = sv[32 * c + 2 * i + 1];
           fma2(x0, x1, cscale, o);
-          if ((i & 7) < kEmuPairsPer8) {
+          if ((i & 7) < emu_pairs_per8<D>()) {
             poly_exp2_2(x0, x1);
           } else {
             x0 = fast_exp2(x0);
@@ -615,23 +743,18 @@ __global__ void __launch_bounds__(320, 1)
           add2(sum0, sum1, x0, x1);
           pk[i] = pack_bf16x2(x0, x1);
         }
-        tmem_st16(stm + 16 * c, pk);
+        tmem_st16(ptm + 16 * c, pk);
       }
       l = l * alpha + (sum0 + sum1);
-      if (j > 0) {
-        ok = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tmem_ld32(otm + c * 32, o);
-            tc_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(otm + c * 32, o);
+          tc_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(otm + c * 32, reinterpret_cast<uint32_t*>(o));
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(otm + c * 32, reinterpret_cast<uint32_t*>(o));
         }
       }
       tc_wait_st();
@@ -691,13 +814,7 @@ __global__ void __launch_bounds__(320, 1)
       bulk_commit();
       bulk_wait_all();
     }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    teardown();
   }
 }
 
@@ -707,11 +824,17 @@ static cudaError_t launch_fwd_d(const CUtensorMap& q, const CUtensorMap& k, cons
   auto fn = fwd_kernel<D>;
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM_ALLOC);
+    // the register split needs the full launch allocation: a smaller one
+    // would leave setmaxnreg.inc waiting, so refuse to launch instead
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  fn<<<grid, 320, FwdCfg<D>::SMEM_ALLOC, stream>>>(q, k, v, o, p);
+  fn<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM_ALLOC, stream>>>(q, k, v, o, p);
   return cudaGetLastError();
 }
 
