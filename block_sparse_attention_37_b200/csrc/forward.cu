@@ -7,17 +7,20 @@
 // for the warpgroups that need it while K and V are loaded once.
 // Roles (384 threads, three aligned warpgroups):
 //   warp 0      TMA producer: both Q tiles, then K/V tiles into a shared ring
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 1      TMEM allocator and tcgen05.mma issuer (whole warp, one
+//               elected lane issues)
 //   warps 2-3   idle (they complete the control warpgroup)
 //   warps 4-7   softmax warpgroup 0 (rows 0..127 of the CTA)
 //   warps 8-11  softmax warpgroup 1 (rows 128..255)
 // The control warpgroup hands registers to the softmax warpgroups
 // (setmaxnreg), which keep a whole 128-key row of S in registers.
-// Tensor memory (512 columns): S/P of warpgroup w at column 128w, O of
-// warpgroup w at 256 + w*D. The MMA warp alternates the two warpgroups, so
-// the tensor core runs one group's PV and next QK^T while the other group's
-// softmax runs (lmnt.cn BSA post, section 3.1: FlashAttention tiles with
-// online softmax over the selected blocks; DiTFastAttnV2 "Fused Kernel").
+// Tensor memory (512 columns), per warpgroup w: S at 128w; d = 64: P at
+// 256 + 64w and O at 384 + 64w (all 512 columns), so the next QK^T may
+// overwrite S while the softmax still works on the row; d = 128: P over S,
+// O at 256 + 128w. The tensor core runs one group's PV and next QK^T while
+// the other group's softmax runs (lmnt.cn BSA post, section 3.1:
+// FlashAttention tiles with online softmax over the selected blocks;
+// DiTFastAttnV2 "Fused Kernel").
 // Output leaves through shared memory and a TMA store.
 #include <utility>
 
@@ -114,53 +117,6 @@ __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
   asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(a) : "l"(a), "l"(b));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
-}
-
-// 2^x on the FMA pipe, two lanes at a time, to take load off the MUFU unit
-// (16 ex2/clk/SM). Range reduction x = j + f with j = round(x) (added to the
-// exponent field) and f in [-0.5, 0.5]; 2^f by a degree-3 polynomial fitted
-// for minimum relative error on that interval (max relative error 7.5e-5,
-// below the bf16 rounding of P). x is clamped at -127, where the result is
-// exactly 0 (see below), so masked (-inf) entries give 0 as on the MUFU path.
-constexpr float kExpC0 = 0.9999280571937561f;
-constexpr float kExpC1 = 0.6932609677314758f;
-constexpr float kExpC2 = 0.2426111400127411f;
-constexpr float kExpC3 = 0.0551716685295105f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
-
-__device__ __forceinline__ void poly_exp2_2(float& x0, float& x1) {
-  x0 = fmaxf(x0, -127.f);
-  x1 = fmaxf(x1, -127.f);
-  uint64_t x, t, j, f, p, c;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c) : "f"(kRoundMagic));
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(t) : "l"(x), "l"(c));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(j) : "l"(t), "l"(c));
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(f) : "l"(x), "l"(j));
-  uint64_t c3, c2, c1, c0;
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c3) : "f"(kExpC3));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c2) : "f"(kExpC2));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c1) : "f"(kExpC1));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(c0) : "f"(kExpC0));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(c3), "l"(f), "l"(c2));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(p) : "l"(p), "l"(f), "l"(c0));
-  uint32_t t0, t1, p0, p1;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(p));
-  p0 = t0 * 8388608u + p0;  // j << 23 added to the exponent bits
-  p1 = t1 * 8388608u + p1;
-  // At x = -127 (every masked key) p(0) = kExpC0 < 1, so the exponent
-  // underflows into the sign bit; the signed max turns that into exactly 0.
-  x0 = __int_as_float(max((int)p0, 0));
-  x1 = __int_as_float(max((int)p1, 0));
-}
-
-// Of every 8 exponent pairs of a row, how many go to the FMA pipe (measured:
-// helps at d = 64 where the softmax dominates, costs at d = 128).
-template <int D>
-__host__ __device__ constexpr int emu_pairs_per8() {
-  return D == 64 ? 2 : 0;
 }
 
 // Fill one group's segment bits from a block-list row.
@@ -517,109 +473,202 @@ __global__ void __launch_bounds__(384, 1)
     }
     } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
-    // The warp serves both warpgroups by polling: whichever QK^T or PV is
-    // ready is issued, so neither warpgroup waits behind the other's barriers.
-    // All 32 lanes run the loop, so its state and the operand descriptors are
-    // warp-uniform; one elected lane issues each MMA and commit.
-    if (T > 0) {
-      auto ready = [&](uint64_t* bar, uint32_t parity) -> bool {
-        return __all_sync(0xffffffffu, mbar_test(smem_u32(bar), parity));
-      };
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      // per-warpgroup state: next tile to QK (T = none), QK^T count, and the
-      // tiles whose PV is outstanding in issue order (f0 first), with their
-      // indices among the warpgroup's tiles
-      struct WgState {
-        int next, cnt, f0, j0, f1, j1;
-        bool q_ok;
-      };
-      auto next_tile = [&](int t, int w) {
-        while (t < T && !((tile_need(sched, nseg, t, act) >> w) & 1)) ++t;
-        return t;
-      };
-      WgState g0{next_tile(0, 0), 0, -1, 0, -1, 0, wg_tiles0 == 0};
-      WgState g1{next_tile(0, 1), 0, -1, 0, -1, 0, wg_tiles1 == 0};
-      // K and V tiles are observed landing in tile order: when tile x is
-      // tested, tile x - S (same stage) is known to have landed and tile
-      // x + S cannot have been loaded (its stage waits for the users of x),
-      // so a one-bit parity test cannot alias another phase of the stage
-      int k_seen = 0, v_seen = 0;
-      // PV of the oldest outstanding tile, if its P and V are ready
-      auto try_pv = [&](WgState& g, int w) -> bool {
-        if (g.f0 < 0) return false;
-        const int u = g.f0, st = u % S;
-        while (v_seen <= u && ready(&v_full[v_seen % S], (uint32_t)(v_seen / S) & 1u)) ++v_seen;
-        if (v_seen <= u || !ready(&p_full[w], (uint32_t)g.j0 & 1u)) return false;
-        tc_fence_after();
-        pv_all(tmem + C::O_COL + w * D, tmem + C::P_COL + w * C::P_STRIDE,
-               smem_desc_sw128(sVa + st * C::TILE, C::CHUNK, 1024), idesc_pv, g.j0 == 0 ? 1u : 0u,
-               std::make_integer_sequence<int, 8>{});
-        tc_commit_warp(&o_ready[w]);
-        tc_commit_warp(&v_empty[2 * st + w]);
-        g.f0 = g.f1;
-        g.j0 = g.j1;
-        g.f1 = -1;
-        return true;
-      };
-      // QK^T of the warpgroup's next tile, if Q, K and the S columns are ready
-      auto try_qk = [&](WgState& g, int w) -> bool {
-        if (g.next >= T || g.f1 >= 0) return false;
-        const int t = g.next, st = t % S;
-        if (!g.q_ok) {
-          if (!ready(&q_full[w], 0u)) return false;
-          g.q_ok = true;
-        }
-        // S is free once the softmax has read it (own P columns) or once the
-        // previous PV is issued (P written over S: the tensor pipe keeps order)
-        const bool s_ok = C::SEP_P ? (g.cnt == 0 || ready(&s_free[w], (uint32_t)(g.cnt - 1) & 1u))
-                                   : (g.f0 < 0);
-        if (!s_ok) return false;
-        while (k_seen <= t && ready(&k_full[k_seen % S], (uint32_t)(k_seen / S) & 1u)) ++k_seen;
-        if (k_seen <= t) return false;
-        tc_fence_after();
-        qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::TILE, 16, 1024),
-               smem_desc_sw128(sKa + st * C::TILE, 16, 1024), idesc_qk, std::make_integer_sequence<int, D / 16>{});
-        tc_commit_warp(&s_full[w]);
-        tc_commit_warp(&k_empty[2 * st + w]);
-        if (g.f0 < 0) {
-          g.f0 = t;
-          g.j0 = g.cnt;
-        } else {
-          g.f1 = t;
-          g.j1 = g.cnt;
-        }
-        ++g.cnt;
-        g.next = next_tile(t + 1, w);
-        return true;
-      };
-      // separate P: the next QK^T first (it unblocks the softmax); shared columns: PV first
-      auto step = [&](WgState& g, int w) -> bool {
-        if (C::SEP_P) {
-          const bool q = try_qk(g, w);
-          return try_pv(g, w) || q;
-        }
-        const bool v = try_pv(g, w);
-        return try_qk(g, w) || v;
-      };
-      uint64_t t_idle = globaltimer_ns();
-      uint32_t spins = 0;
-      while (g0.next < T || g0.f0 >= 0 || g1.next < T || g1.f0 >= 0) {
-        const bool a0 = step(g0, 0);
-        const bool a1 = step(g1, 1);
-        if (a0 || a1) {
-          spins = 0;
-          continue;
-        }
-        if ((++spins & 63u) == 0) {
-          const uint64_t now = __shfl_sync(0xffffffffu, globaltimer_ns(), 0);
-          if (spins == 64) t_idle = now;
-          if (__any_sync(0xffffffffu, *abort_flag != 0) || now - t_idle > kWaitLimitNs) {
-            cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
-            break;
+    // Two issue strategies, chosen by what measured faster for each layout.
+    if constexpr (C::SEP_P) {
+      // The warp serves both warpgroups by polling: whichever QK^T or PV is
+      // ready is issued, so neither warpgroup waits behind the other's barriers.
+      // All 32 lanes run the loop, so its state and the operand descriptors are
+      // warp-uniform; one elected lane issues each MMA and commit.
+      if (T > 0) {
+        auto ready = [&](uint64_t* bar, uint32_t parity) -> bool {
+          return __all_sync(0xffffffffu, mbar_test(smem_u32(bar), parity));
+        };
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+        // per-warpgroup state: next tile to QK (T = none), QK^T count, and the
+        // tiles whose PV is outstanding in issue order (f0 first), with their
+        // indices among the warpgroup's tiles
+        struct WgState {
+          int next, cnt, f0, j0, f1, j1;
+          bool q_ok;
+        };
+        auto next_tile = [&](int t, int w) {
+          while (t < T && !((tile_need(sched, nseg, t, act) >> w) & 1)) ++t;
+          return t;
+        };
+        WgState g0{next_tile(0, 0), 0, -1, 0, -1, 0, wg_tiles0 == 0};
+        WgState g1{next_tile(0, 1), 0, -1, 0, -1, 0, wg_tiles1 == 0};
+        // K and V tiles are observed landing in tile order: when tile x is
+        // tested, tile x - S (same stage) is known to have landed and tile
+        // x + S cannot have been loaded (its stage waits for the users of x),
+        // so a one-bit parity test cannot alias another phase of the stage
+        int k_seen = 0, v_seen = 0;
+        // PV of the oldest outstanding tile, if its P and V are ready
+        auto try_pv = [&](WgState& g, int w) -> bool {
+          if (g.f0 < 0) return false;
+          const int u = g.f0, st = u % S;
+          while (v_seen <= u && ready(&v_full[v_seen % S], (uint32_t)(v_seen / S) & 1u)) ++v_seen;
+          if (v_seen <= u || !ready(&p_full[w], (uint32_t)g.j0 & 1u)) return false;
+          tc_fence_after();
+          pv_all(tmem + C::O_COL + w * D, tmem + C::P_COL + w * C::P_STRIDE,
+                 smem_desc_sw128(sVa + st * C::TILE, C::CHUNK, 1024), idesc_pv, g.j0 == 0 ? 1u : 0u,
+                 std::make_integer_sequence<int, 8>{});
+          tc_commit_warp(&o_ready[w]);
+          tc_commit_warp(&v_empty[2 * st + w]);
+          g.f0 = g.f1;
+          g.j0 = g.j1;
+          g.f1 = -1;
+          return true;
+        };
+        // QK^T of the warpgroup's next tile, if Q, K and the S columns are ready
+        auto try_qk = [&](WgState& g, int w) -> bool {
+          if (g.next >= T || g.f1 >= 0) return false;
+          const int t = g.next, st = t % S;
+          if (!g.q_ok) {
+            if (!ready(&q_full[w], 0u)) return false;
+            g.q_ok = true;
+          }
+          // S is free once the softmax has read it (own P columns) or once the
+          // previous PV is issued (P written over S: the tensor pipe keeps order)
+          const bool s_ok = C::SEP_P ? (g.cnt == 0 || ready(&s_free[w], (uint32_t)(g.cnt - 1) & 1u))
+                                     : (g.f0 < 0);
+          if (!s_ok) return false;
+          while (k_seen <= t && ready(&k_full[k_seen % S], (uint32_t)(k_seen / S) & 1u)) ++k_seen;
+          if (k_seen <= t) return false;
+          tc_fence_after();
+          qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::TILE, 16, 1024),
+                 smem_desc_sw128(sKa + st * C::TILE, 16, 1024), idesc_qk, std::make_integer_sequence<int, D / 16>{});
+          tc_commit_warp(&s_full[w]);
+          tc_commit_warp(&k_empty[2 * st + w]);
+          if (g.f0 < 0) {
+            g.f0 = t;
+            g.j0 = g.cnt;
+          } else {
+            g.f1 = t;
+            g.j1 = g.cnt;
+          }
+          ++g.cnt;
+          g.next = next_tile(t + 1, w);
+          return true;
+        };
+        // separate P: the next QK^T first (it unblocks the softmax); shared columns: PV first
+        auto step = [&](WgState& g, int w) -> bool {
+          if (C::SEP_P) {
+            const bool q = try_qk(g, w);
+            return try_pv(g, w) || q;
+          }
+          const bool v = try_pv(g, w);
+          return try_qk(g, w) || v;
+        };
+        uint64_t t_idle = globaltimer_ns();
+        uint32_t spins = 0;
+        while (g0.next < T || g0.f0 >= 0 || g1.next < T || g1.f0 >= 0) {
+          const bool a0 = step(g0, 0);
+          const bool a1 = step(g1, 1);
+          if (a0 || a1) {
+            spins = 0;
+            continue;
+          }
+          if ((++spins & 63u) == 0) {
+            const uint64_t now = __shfl_sync(0xffffffffu, globaltimer_ns(), 0);
+            if (spins == 64) t_idle = now;
+            if (__any_sync(0xffffffffu, *abort_flag != 0) || now - t_idle > kWaitLimitNs) {
+              cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+              break;
+            }
           }
         }
+      }
+    } else {
+      // Fixed issue order with blocking (suspending) waits, per tile t:
+      // QK^T(t) of each warpgroup that needs t, then the PV of each such
+      // warpgroup's previous tile. With separate P columns QK^T(t) waits only
+      // for S to be read, so it overlaps the softmax of the previous tile; with
+      // P written over S the PV goes first. All 32 lanes run the loop, so its
+      // state and the operand descriptors are warp-uniform; one elected lane
+      // issues each MMA and commit.
+      if (T > 0) {
+        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
+        auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+          return warp_all(mbar_wait(bar, parity, abort_flag));
+        };
+        // per warpgroup: tile whose PV is outstanding (-1: none) and its index
+        // among the warpgroup's tiles; QK^T issued so far
+        int pt0 = -1, pj0 = 0, pt1 = -1, pj1 = 0, c0 = 0, c1 = 0;
+        bool q0 = false, q1 = false;
+        // V tiles are observed in tile order (K tiles are, by the loop), so a
+        // one-bit parity test never aliases another phase of a shared stage:
+        // when tile x is waited for, tile x - S has landed, and tile x + S
+        // cannot have been loaded before this warp released x
+        int v_seen = 0;
+        auto pv = [&](int w) -> bool {
+          const int u = w ? pt1 : pt0, jj = w ? pj1 : pj0;
+          for (; v_seen <= u; ++v_seen)
+            if (!wwait(&v_full[v_seen % S], (uint32_t)(v_seen / S) & 1u)) return false;
+          if (!wwait(&p_full[w], (uint32_t)jj & 1u)) return false;
+          tc_fence_after();
+          pv_all(tmem + C::O_COL + w * D, tmem + C::P_COL + w * C::P_STRIDE,
+                 smem_desc_sw128(sVa + (u % S) * C::TILE, C::CHUNK, 1024), idesc_pv, jj == 0 ? 1u : 0u,
+                 std::make_integer_sequence<int, 8>{});
+          tc_commit_warp(&o_ready[w]);
+          tc_commit_warp(&v_empty[2 * (u % S) + w]);
+          (w ? pt1 : pt0) = -1;
+          return true;
+        };
+        auto qk = [&](int w, int t) -> bool {
+          bool& q = w ? q1 : q0;
+          if (!q) {
+            if (!wwait(&q_full[w], 0u)) return false;
+            q = true;
+          }
+          const int c = w ? c1 : c0;
+          if (C::SEP_P) {
+            if (c > 0 && !wwait(&s_free[w], (uint32_t)(c - 1) & 1u)) return false;
+          } else if ((w ? pt1 : pt0) >= 0 && !pv(w)) {
+            return false;
+          }
+          tc_fence_after();
+          qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::TILE, 16, 1024),
+                 smem_desc_sw128(sKa + (t % S) * C::TILE, 16, 1024), idesc_qk,
+                 std::make_integer_sequence<int, D / 16>{});
+          tc_commit_warp(&s_full[w]);
+          tc_commit_warp(&k_empty[2 * (t % S) + w]);
+          return true;
+        };
+        // outstanding PVs of tiles below `limit`, oldest first (a younger
+        // one's V can depend on the older one's release)
+        auto flush_below = [&](int limit) -> bool {
+          const bool f0 = pt0 >= 0 && pt0 < limit, f1 = pt1 >= 0 && pt1 < limit;
+          if (f0 && f1 && pt1 < pt0) return pv(1) && pv(0);
+          return (!f0 || pv(0)) && (!f1 || pv(1));
+        };
+        bool ok = true;
+        for (int t = 0; t < T && ok; ++t) {
+          // K(t) arrives only after the producer has reloaded V for tile t - 1,
+          // which needs every PV of tile t - 1 - S: issue those first
+          ok = flush_below(t - S) && wwait(&k_full[t % S], (uint32_t)(t / S) & 1u);
+          if (!ok) break;
+          const int nw = tile_need(sched, nseg, t, act);
+          if (nw & 1) ok = qk(0, t);
+          if (ok && (nw & 2)) ok = qk(1, t);
+          if (C::SEP_P) {
+            if (ok && (nw & 1) && pt0 >= 0) ok = pv(0);
+            if (ok && (nw & 2) && pt1 >= 0) ok = pv(1);
+          }
+          if (nw & 1) {
+            pt0 = t;
+            pj0 = c0++;
+          }
+          if (nw & 2) {
+            pt1 = t;
+            pj1 = c1++;
+          }
+        }
+        ok = ok && flush_below(T);
+        if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
       }
     }
     }
@@ -734,12 +783,8 @@ __global__ void __launch_bounds__(384, 1)
         for (int i = 0; i < 16; ++i) {
           float x0 = sv[32 * c + 2 * i], x1 = sv[32 * c + 2 * i + 1];
           fma2(x0, x1, cscale, o);
-          if ((i & 7) < emu_pairs_per8<D>()) {
-            poly_exp2_2(x0, x1);
-          } else {
-            x0 = fast_exp2(x0);
-            x1 = fast_exp2(x1);
-          }
+          x0 = fast_exp2(x0);
+          x1 = fast_exp2(x1);
           add2(sum0, sum1, x0, x1);
           pk[i] = pack_bf16x2(x0, x1);
         }
