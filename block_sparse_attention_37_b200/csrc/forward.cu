@@ -119,49 +119,14 @@ __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
   asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
 }
 
-// Fill one group's segment bits from a block-list row.
-__device__ void fill_group_bits(const AttnParams& p, size_t row, uint32_t* vb, uint32_t* pb, int lane) {
-  const int spb = p.block_k >> 6;
-  int n = p.cnt[row];
-  if (n < 0 || n > p.max_k) {
-    if (lane == 0) record_error(BSA_DEVERR_BAD_INDEX);
-    n = n < 0 ? 0 : p.max_k;
-  }
-  const int32_t* ip = p.idx + row * p.max_k;
-  const uint8_t* fp = p.flag + row * p.max_k;
-  for (int e = lane; e < n; e += 32) {
-    const int J = ip[e];
-    if (J < 0 || J >= p.nKB) {
-      record_error(BSA_DEVERR_BAD_INDEX);
-      continue;
-    }
-    bool part = fp[e] == BSA_BLOCK_PARTIAL;
-    if (part && !p.has_gna) {
-      record_error(BSA_DEVERR_NO_GEOMETRY);
-      part = false;
-    }
-    for (int u = 0; u < spb; ++u) {
-      const int s = J * spb + u;
-      if (s >= p.nSeg) break;
-      atomicOr(&vb[s >> 5], 1u << (s & 31));
-      if (part) atomicOr(&pb[s >> 5], 1u << (s & 31));
-    }
-  }
-}
-
 // Sorted union schedule of the CTA's four 64-row groups (warp 0). Returns count.
+// Warp-parallel throughout: the block-list rows of all groups are read in one
+// round of loads, and segments are emitted 32 at a time by ballot compaction.
 __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0, uint32_t* vb,
                                  uint32_t* pb, int32_t* sched, int lane) {
   const int nwords = (p.nSeg + 31) >> 5;
   for (int w = lane; w < 5 * 64; w += 32) vb[w] = 0u;  // vb[4][64] then pb[64]
   __syncwarp();
-  bool valid[4];
-  int I[4];
-#pragma unroll
-  for (int g = 0; g < 4; ++g) {
-    valid[g] = row0 + 64 * g < p.N;
-    I[g] = valid[g] ? (row0 + 64 * g) / p.block_q : -1;
-  }
   const int spb = p.block_k >> 6;
   if (mode == BSA_HEAD_FULL) {
     for (int w = lane; w < nwords; w += 32) vb[w] = bit_range(0, min(32, p.nSeg - w * 32));
@@ -180,56 +145,124 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
     if (p.cnt == nullptr) {
       if (lane == 0) record_error(BSA_DEVERR_BAD_INDEX);
     } else {
-#pragma unroll
-      for (int g = 0; g < 4; ++g)
-        if (valid[g] && (g == 0 || I[g] != I[g - 1]))
-          fill_group_bits(p, (size_t)bh * p.nQB + I[g], vb + g * 64, pb, lane);
+      // lane g < 4: entries of group g's block-list row; 0 when the group is
+      // past N or shares its predecessor's query block (it copies them below)
+      int n_l = 0;
+      if (lane < 4) {
+        const int rq = row0 + 64 * lane;
+        const int Ig = rq / p.block_q;
+        if (rq < p.N && (lane == 0 || Ig != (rq - 64) / p.block_q)) {
+          n_l = p.cnt[(size_t)bh * p.nQB + Ig];
+          if (n_l < 0 || n_l > p.max_k) {
+            record_error(BSA_DEVERR_BAD_INDEX);
+            n_l = n_l < 0 ? 0 : p.max_k;
+          }
+        }
+      }
+      const int n0 = __shfl_sync(0xffffffffu, n_l, 0), n1 = __shfl_sync(0xffffffffu, n_l, 1);
+      const int n2 = __shfl_sync(0xffffffffu, n_l, 2), n3 = __shfl_sync(0xffffffffu, n_l, 3);
+      const int e1 = n0, e2 = n0 + n1, e3 = n0 + n1 + n2, tot = e3 + n3;
+      for (int e = lane; e < tot; e += 32) {
+        const int g = e < e1 ? 0 : e < e2 ? 1 : e < e3 ? 2 : 3;
+        const int k = e - (g == 0 ? 0 : g == 1 ? e1 : g == 2 ? e2 : e3);
+        const size_t at = ((size_t)bh * p.nQB + (row0 + 64 * g) / p.block_q) * p.max_k + k;
+        const int J = p.idx[at];
+        if (J < 0 || J >= p.nKB) {
+          record_error(BSA_DEVERR_BAD_INDEX);
+          continue;
+        }
+        bool part = p.flag[at] == BSA_BLOCK_PARTIAL;
+        if (part && !p.has_gna) {
+          record_error(BSA_DEVERR_NO_GEOMETRY);
+          part = false;
+        }
+        for (int u = 0; u < spb; ++u) {
+          const int s = J * spb + u;
+          if (s >= p.nSeg) break;
+          atomicOr(&vb[g * 64 + (s >> 5)], 1u << (s & 31));
+          if (part) atomicOr(&pb[s >> 5], 1u << (s & 31));
+        }
+      }
     }
     __syncwarp();
     // groups sharing a query block share its bits; groups past N copy their neighbour
     for (int g = 1; g < 4; ++g) {
-      if (!valid[g] || I[g] == I[g - 1])
+      const int rq = row0 + 64 * g;
+      if (rq >= p.N || rq / p.block_q == (rq - 64) / p.block_q)
         for (int w = lane; w < 64; w += 32) vb[g * 64 + w] = vb[(g - 1) * 64 + w];
       __syncwarp();
     }
   }
   __syncwarp();
-  const int w0 = lane, w1 = lane + 32;
-  uint32_t a0 = 0u, a1 = 0u;
-  if (w0 < nwords) a0 = vb[w0] | vb[64 + w0] | vb[128 + w0] | vb[192 + w0];
-  if (w1 < nwords) a1 = vb[w1] | vb[64 + w1] | vb[128 + w1] | vb[192 + w1];
-  const int c0 = __popc(a0), c1 = __popc(a1);
-  int i0 = c0, i1 = c1;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int t0 = __shfl_up_sync(0xffffffffu, i0, o);
-    const int t1 = __shfl_up_sync(0xffffffffu, i1, o);
-    if (lane >= o) {
-      i0 += t0;
-      i1 += t1;
+  // emit the kept segments in ascending order, 32 at a time
+  int base = 0;
+  for (int s0 = 0; s0 < p.nSeg; s0 += 32) {
+    const int wd = s0 >> 5, s = s0 + lane;
+    const uint32_t v0 = vb[wd], v1 = vb[64 + wd], v2 = vb[128 + wd], v3 = vb[192 + wd], pw = pb[wd];
+    const uint32_t gb = ((v0 >> lane) & 1u) | (((v1 >> lane) & 1u) << 1) | (((v2 >> lane) & 1u) << 2) |
+                        (((v3 >> lane) & 1u) << 3);
+    const bool keep = s < p.nSeg && gb != 0u;
+    const uint32_t bal = __ballot_sync(0xffffffffu, keep);
+    if (keep)
+      sched[base + __popc(bal & ((1u << lane) - 1u))] =
+          s | (int)(gb << kGrpShift) | (((pw >> lane) & 1u) ? kPart4 : 0);
+    base += __popc(bal);
+  }
+  return base;
+}
+
+// Work order of the grid (longest first, so no long CTA starts late): all
+// FULL heads, then the SPARSE heads by query pair (pair 0 of every sparse
+// head first: the text rows lead the sequence and keep every key), then
+// the SKIP heads. A bijection from blockIdx.x onto the B*H*nQP (b, h, pair)
+// items; heads with an invalid mode count as sparse (their CTA reports it).
+// Run by a whole warp; every warp computes the same answer.
+__device__ __forceinline__ void map_item(const AttnParams& p, int nQP, int lane, int& bh, int& pair) {
+  int nF = 0, nK = 0;
+  for (int h0 = 0; h0 < p.H; h0 += 32) {
+    const int hh = h0 + lane;
+    const int md = hh < p.H ? p.head_mode[hh] : -1;
+    nF += __popc(__ballot_sync(0xffffffffu, md == BSA_HEAD_FULL));
+    nK += __popc(__ballot_sync(0xffffffffu, md == BSA_HEAD_SKIP));
+  }
+  const int nS = p.H - nF - nK;
+  const int k = (int)blockIdx.x;
+  const int perF = p.B * nF * nQP, perS = p.B * nS * nQP;
+  int cls, b, m;
+  if (k < perF) {
+    cls = BSA_HEAD_FULL;
+    pair = k % nQP;
+    b = (k / nQP) / nF;
+    m = (k / nQP) % nF;
+  } else if (k < perF + perS) {
+    const int r = k - perF;
+    cls = BSA_HEAD_SPARSE;
+    pair = r / (p.B * nS);
+    b = (r % (p.B * nS)) / nS;
+    m = (r % (p.B * nS)) % nS;
+  } else {
+    const int r = k - perF - perS;
+    cls = BSA_HEAD_SKIP;
+    pair = r % nQP;
+    b = (r / nQP) / nK;
+    m = (r / nQP) % nK;
+  }
+  int h = 0;
+  for (int h0 = 0; h0 < p.H; h0 += 32) {
+    const int hh = h0 + lane;
+    const int md = hh < p.H ? p.head_mode[hh] : -1;
+    const bool in = hh < p.H && (cls == BSA_HEAD_SPARSE ? (md != BSA_HEAD_FULL && md != BSA_HEAD_SKIP) : md == cls);
+    const uint32_t mask = __ballot_sync(0xffffffffu, in);
+    const int c = __popc(mask);
+    if (m < c) {  // the m-th set bit of mask
+      uint32_t mm = mask;
+      for (int i = 0; i < m; ++i) mm &= mm - 1u;
+      h = h0 + __ffs((int)mm) - 1;
+      break;
     }
+    m -= c;
   }
-  const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
-  const int tot1 = __shfl_sync(0xffffffffu, i1, 31);
-  int off = i0 - c0;
-  for (uint32_t a = a0; a; a &= a - 1) {
-    const int b = __ffs(a) - 1;
-    int e = w0 * 32 + b;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) e |= ((vb[g * 64 + w0] >> b) & 1u) << (kGrpShift + g);
-    if ((pb[w0] >> b) & 1u) e |= kPart4;
-    sched[off++] = e;
-  }
-  off = tot0 + i1 - c1;
-  for (uint32_t a = a1; a; a &= a - 1) {
-    const int b = __ffs(a) - 1;
-    int e = w1 * 32 + b;
-#pragma unroll
-    for (int g = 0; g < 4; ++g) e |= ((vb[g * 64 + w1] >> b) & 1u) << (kGrpShift + g);
-    if ((pb[w1] >> b) & 1u) e |= kPart4;
-    sched[off++] = e;
-  }
-  return tot0 + tot1;
+  bh = b * p.H + h;
 }
 
 // Bit w of the result: does warpgroup w need tile t?
@@ -298,8 +331,8 @@ __global__ void __launch_bounds__(384, 1)
                                              ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nQP = (p.N + 255) >> 8;
-  const int pair = (int)blockIdx.x % nQP;
-  const int bh = (int)blockIdx.x / nQP;
+  int bh, pair;
+  map_item(p, nQP, lane, bh, pair);
   const int h = bh % p.H;
   const int row0 = pair * 256;
 
@@ -349,6 +382,19 @@ __global__ void __launch_bounds__(384, 1)
     }
     misc[1] = 0;
     fence_barrier_init();
+    // Q does not depend on the key schedule: both tiles are loaded now and
+    // land while warp 0 builds it (rows past N read as zeros)
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      mbar_arrive_expect_tx(&q_full[w], C::TILE);
+      for (int c = 0; c < D / 64; ++c)
+        for (int h2 = 0; h2 < 2; ++h2)
+          tma_load_3d(sQ + w * C::TILE + c * C::CHUNK + h2 * (C::CHUNK / 2), &tmQ, &q_full[w], c * 64,
+                      row0 + 128 * w + 64 * h2, bh);
+    }
   }
   if (warp == 1) {
     tmem_alloc(misc, 512);
@@ -401,18 +447,6 @@ __global__ void __launch_bounds__(384, 1)
     if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0 && T > 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-#pragma unroll
-      for (int w = 0; w < 2; ++w) {
-        if ((w ? wg_tiles1 : wg_tiles0) == 0) continue;
-        mbar_arrive_expect_tx(&q_full[w], C::TILE);
-        for (int c = 0; c < D / 64; ++c)
-          for (int r = 0; r < 2; ++r)
-            tma_load_3d(sQ + w * C::TILE + c * C::CHUNK + r * (C::CHUNK / 2), &tmQ, &q_full[w], c * 64,
-                        row0 + 128 * w + 64 * r, bh);
-      }
       int k_issued = 0, v_issued = 0;
       uint32_t kpar = 0u, vpar = 0u;  // phase parity per (stage, warpgroup) release barrier
       for (int t = 0; t < T; ++t) {
@@ -463,13 +497,17 @@ __global__ void __launch_bounds__(384, 1)
           while (!mbar_try_wait(smem_u32(bar), ph) && globaltimer_ns() - t0 < kWaitLimitNs) {
           }
         };
-        if (wg_tiles0 > 0) drain(&q_full[0], 0u);
-        if (wg_tiles1 > 0) drain(&q_full[1], 0u);
         for (int t = k_issued - S < 0 ? 0 : k_issued - S; t < k_issued; ++t)
           drain(&k_full[t % S], (uint32_t)(t / S) & 1u);
         for (int t = v_issued - S < 0 ? 0 : v_issued - S; t < v_issued; ++t)
           drain(&v_full[t % S], (uint32_t)(t / S) & 1u);
       }
+    }
+    if (lane == 0) {  // every CTA loaded Q: it must have landed before the CTA ends
+      const uint64_t t0 = globaltimer_ns();
+      for (int w = 0; w < 2; ++w)
+        while (!mbar_try_wait(smem_u32(&q_full[w]), 0u) && globaltimer_ns() - t0 < kWaitLimitNs) {
+        }
     }
     } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -810,6 +848,9 @@ __global__ void __launch_bounds__(384, 1)
     if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
 
     // ---------------------------------------------------------------- epilogue
+    // O is staged over the Q tile: a warpgroup that computed nothing has not
+    // seen Q land yet
+    if (j == 0 && !warp_all(mbar_wait(&q_full[w], 0u, abort_flag))) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
     bool have = ok && j > 0;
     if (have) {
       have = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
