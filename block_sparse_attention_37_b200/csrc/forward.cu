@@ -93,7 +93,9 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* s
       : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// The staged tile may be reused (or the CTA end) once the copies have read
+// it; their global writes complete before the grid does.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
@@ -212,12 +214,10 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
 }
 
 // Work order of the grid (longest first, so no long CTA starts late): all
-// FULL heads, then the SPARSE heads by query pair (pair 0 of every sparse
-// head first: the text rows lead the sequence and keep every key), then
-// the SKIP heads. A bijection from blockIdx.x onto the B*H*nQP (b, h, pair)
+// FULL heads, then the SPARSE heads (below), then the SKIP heads. A bijection from blockIdx.x onto the B*H*nQP (b, h, pair)
 // items; heads with an invalid mode count as sparse (their CTA reports it).
 // Run by a whole warp; every warp computes the same answer.
-__device__ __forceinline__ void map_item(const AttnParams& p, int nQP, int lane, int& bh, int& pair) {
+__device__ __forceinline__ void map_item(const AttnParams& p, int d, int nQP, int lane, int& bh, int& pair) {
   int nF = 0, nK = 0;
   for (int h0 = 0; h0 < p.H; h0 += 32) {
     const int hh = h0 + lane;
@@ -235,11 +235,22 @@ __device__ __forceinline__ void map_item(const AttnParams& p, int nQP, int lane,
     b = (k / nQP) / nF;
     m = (k / nQP) % nF;
   } else if (k < perF + perS) {
+    // (b, sparse head) units in chunks whose K and V fit in a quarter of L2
+    // (32 MiB; measured: chunks near half of L2 thrash), query pair by query
+    // pair within a chunk: the dense text rows (pair 0) go first while the
+    // K/V the chunk's CTAs share stay cached
     const int r = k - perF;
+    const int units = p.B * nS;
+    const long long fit = (32ll << 20) / (4ll * p.N * d);
+    const int G = (int)(fit < 1 ? 1 : fit > units ? units : fit);
+    const int c = r / (G * nQP);
+    const int gsz = min(G, units - c * G);
+    const int rr = r - c * G * nQP;
+    const int u = c * G + rr % gsz;
     cls = BSA_HEAD_SPARSE;
-    pair = r / (p.B * nS);
-    b = (r % (p.B * nS)) / nS;
-    m = (r % (p.B * nS)) % nS;
+    pair = rr / gsz;
+    b = u / nS;
+    m = u % nS;
   } else {
     const int r = k - perF - perS;
     cls = BSA_HEAD_SKIP;
@@ -247,8 +258,9 @@ __device__ __forceinline__ void map_item(const AttnParams& p, int nQP, int lane,
     b = (r / nQP) / nK;
     m = (r / nQP) % nK;
   }
-  int h = 0;
-  for (int h0 = 0; h0 < p.H; h0 += 32) {
+  int h = m;  // every head in one class: the m-th head is head m
+  const int ncls = cls == BSA_HEAD_FULL ? nF : cls == BSA_HEAD_SKIP ? nK : nS;
+  for (int h0 = 0; ncls < p.H && h0 < p.H; h0 += 32) {
     const int hh = h0 + lane;
     const int md = hh < p.H ? p.head_mode[hh] : -1;
     const bool in = hh < p.H && (cls == BSA_HEAD_SPARSE ? (md != BSA_HEAD_FULL && md != BSA_HEAD_SKIP) : md == cls);
@@ -332,7 +344,7 @@ __global__ void __launch_bounds__(384, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nQP = (p.N + 255) >> 8;
   int bh, pair;
-  map_item(p, nQP, lane, bh, pair);
+  map_item(p, D, nQP, lane, bh, pair);
   const int h = bh % p.H;
   const int row0 = pair * 256;
 
@@ -898,7 +910,7 @@ __global__ void __launch_bounds__(384, 1)
             tma_store_3d(&tmO, stage + c * C::CHUNK + rr * (C::CHUNK / 2), c * 64, row0 + 128 * w + 64 * rr,
                          bh);
       bulk_commit();
-      bulk_wait_all();
+      bulk_wait_read();
     }
     teardown();
   }
