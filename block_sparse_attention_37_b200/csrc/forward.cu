@@ -235,20 +235,30 @@ __device__ __forceinline__ void map_item(const AttnParams& p, int d, int nQP, in
     b = (k / nQP) / nF;
     m = (k / nQP) % nF;
   } else if (k < perF + perS) {
-    // (b, sparse head) units in chunks whose K and V fit in a quarter of L2
-    // (32 MiB; measured: chunks near half of L2 thrash), query pair by query
-    // pair within a chunk: the dense text rows (pair 0) go first while the
-    // K/V the chunk's CTAs share stay cached
-    const int r = k - perF;
+    // pair 0 of every (b, sparse head) unit first: the text rows lead the
+    // sequence and keep every key, so these are the longest sparse CTAs.
+    // The other pairs follow in chunks of units whose K and V fit in a
+    // quarter of L2 (32 MiB; measured: chunks near half of L2 thrash),
+    // query pair by query pair within a chunk, so the K/V the chunk's CTAs
+    // share stay cached.
+    int r = k - perF;
     const int units = p.B * nS;
-    const long long fit = (32ll << 20) / (4ll * p.N * d);
-    const int G = (int)(fit < 1 ? 1 : fit > units ? units : fit);
-    const int c = r / (G * nQP);
-    const int gsz = min(G, units - c * G);
-    const int rr = r - c * G * nQP;
-    const int u = c * G + rr % gsz;
     cls = BSA_HEAD_SPARSE;
-    pair = rr / gsz;
+    int u;
+    if (r < units) {
+      pair = 0;
+      u = r;
+    } else {
+      r -= units;
+      const int np = nQP - 1;  // pairs 1 .. nQP-1 (np >= 1 here)
+      const long long fit = (32ll << 20) / (4ll * p.N * d);
+      const int G = (int)(fit < 1 ? 1 : fit > units ? units : fit);
+      const int c = r / (G * np);
+      const int gsz = min(G, units - c * G);
+      const int rr = r - c * G * np;
+      u = c * G + rr % gsz;
+      pair = 1 + rr / gsz;
+    }
     b = u / nS;
     m = u % nS;
   } else {
