@@ -16,7 +16,7 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libbsa.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE, ERR_INFEASIBLE = range(7)
 DEVERR_NONE, DEVERR_BAD_INDEX, DEVERR_TIMEOUT, DEVERR_SCHEDULE, DEVERR_NO_GEOMETRY = range(5)
 HEAD_FULL, HEAD_SPARSE, HEAD_SKIP = 0, 1, 2
 BLOCK_NONE, BLOCK_FULL, BLOCK_PARTIAL = 0, 1, 2
@@ -26,7 +26,8 @@ SELECT_POOLED_QK, SELECT_FULL_SCORE = 1, 2
 EXPORTS = (
     "bsa_version", "bsa_error_string", "bsa_build_mask", "bsa_select_workspace_size",
     "bsa_select_topk", "bsa_forward", "bsa_gna_tiled_len", "bsa_permute_tiles",
-    "bsa_unpermute_tiles", "bsa_get_device_error", "bsa_select_topk_static",
+    "bsa_unpermute_tiles", "bsa_get_device_error", "bsa_select_topk_static", "bsa_rse",
+    "bsa_plan_heads",
 )
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -104,6 +105,9 @@ def _lib():
         lib.bsa_unpermute_tiles.argtypes = [P, P, ctypes.c_int32, P, P, P]
         lib.bsa_get_device_error.argtypes = [P, P]
         lib.bsa_select_topk_static.argtypes = [P, P, P, P, P, P, P]
+        lib.bsa_rse.argtypes = [P, P, P, P, P]
+        lib.bsa_plan_heads.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, ctypes.c_double,
+                                       P, P]
         _LIB = lib
     return _LIB
 
@@ -252,6 +256,30 @@ def permute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
 def unpermute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
     _check(_lib().bsa_unpermute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), _ptr_array(ins, "in"),
                                       _ptr_array(outs, "out"), _stream(stream)), "bsa_unpermute_tiles")
+
+
+def rse(dm: Dims, y_m, y_o, out, stream=None):
+    """bsa_rse: out (cuda float64 [4*H]) receives I(h) then the three sums per head."""
+    if out.dtype != torch.float64 or not out.is_cuda or out.numel() < 4 * dm.H:
+        raise ValueError("out must be a cuda float64 tensor of 4*H elements")
+    _check(_lib().bsa_rse(ctypes.byref(dm), _ptr(y_m, torch.bfloat16, "y_m"), _ptr(y_o, torch.bfloat16, "y_o"),
+                          ctypes.c_void_p(out.data_ptr()), _stream(stream)), "bsa_rse")
+
+
+def plan_heads(rse_hm, cost_hm, delta: float, c: float = 1.5):
+    """bsa_plan_heads on host arrays [H, M]; returns (choice int32 [H], total cost)."""
+    import numpy as np
+    r = np.ascontiguousarray(rse_hm, dtype=np.float64)
+    k = np.ascontiguousarray(cost_hm, dtype=np.int64)
+    if r.ndim != 2 or r.shape != k.shape:
+        raise ValueError("rse and cost must both be [H, M]")
+    H, M = r.shape
+    choice = np.zeros(H, dtype=np.int32)
+    total = ctypes.c_int64(0)
+    _check(_lib().bsa_plan_heads(H, M, r.ctypes.data_as(ctypes.c_void_p), k.ctypes.data_as(ctypes.c_void_p),
+                                 float(delta), float(c), choice.ctypes.data_as(ctypes.c_void_p),
+                                 ctypes.byref(total)), "bsa_plan_heads")
+    return choice, int(total.value)
 
 
 def get_device_error(stream=None) -> int:

@@ -148,6 +148,7 @@ const char* bsa_error_string(int status) {
     case BSA_ERR_WORKSPACE: return "workspace missing or too small";
     case BSA_ERR_CUDA: return "CUDA error";
     case BSA_ERR_DEVICE: return "device-side fault recorded";
+    case BSA_ERR_INFEASIBLE: return "no plan meets the error budget";
     default: return "unknown status";
   }
 }

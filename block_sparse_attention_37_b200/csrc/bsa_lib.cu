@@ -7,3 +7,4 @@
 #include "permute.cu"
 #include "select.cu"
 #include "select_static.cu"
+#include "plan.cu"

@@ -2,8 +2,10 @@
  * bsa.h - block-sparse attention for diffusion transformers on B200 (sm_100a).
  *
  * A small C ABI over hand-written CUDA kernels. Every pointer argument named
- * "device" is caller-owned device memory; the library never allocates, never
- * synchronises the host (except bsa_get_device_error) and has no CPU fallback.
+ * "device" is caller-owned device memory; the library never allocates device
+ * memory, never synchronises the host (except bsa_get_device_error) and has
+ * no CPU fallback. The one host-only routine, bsa_plan_heads, works on host
+ * arrays.
  * All launches are asynchronous on the caller's stream, passed as `void*`
  * holding a cudaStream_t (NULL = legacy default stream).
  *
@@ -34,6 +36,7 @@ extern "C" {
 #define BSA_ERR_WORKSPACE 3    /* workspace missing or smaller than required   */
 #define BSA_ERR_CUDA 4         /* a CUDA runtime/driver call failed            */
 #define BSA_ERR_DEVICE 5       /* a kernel recorded a fault (see below)        */
+#define BSA_ERR_INFEASIBLE 6   /* no plan meets the error budget               */
 
 /* device error word values (bsa_get_device_error) */
 #define BSA_DEVERR_NONE 0
@@ -221,6 +224,39 @@ int bsa_permute_tiles(const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_
                       const void* const* in, void* const* out, void* stream);
 int bsa_unpermute_tiles(const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_tensors,
                         const void* const* in, void* const* out, void* stream);
+
+/* bsa_rse: the single-layer relative squared error of a compressed output,
+ * per head (DiTFastAttnV2, "efficient compression plan search"):
+ *   I(h) = sum (y_m - y_o)^2 / sum (y_o - mean(y_o))^2
+ * with the sums over head h's outputs of every batch item, token and channel
+ * (the printed numerator subtracts mean(y_o); read as y_m - y_o).
+ *  dims: B, H, N and d are read (block sizes and n_text are ignored).
+ *  y_m, y_o: device bf16 [B, H, N, d]: the output under a method m and the
+ *    uncompressed output of the same layer and inputs.
+ *  out: device double [4 * H], caller-owned, overwritten: out[h] = I(h);
+ *    out[H + 3h + 0..2] = sum (y_m - y_o)^2, sum y_o, sum y_o^2 (fp64).
+ *    A head whose y_o is constant has a zero denominator (I = inf or NaN).
+ *  Errors: INVALID_ARG (null pointer, bad dims), UNSUPPORTED (N*d not a
+ *  multiple of 8), CUDA. */
+int bsa_rse(const bsa_dims* dims, const void* y_m, const void* y_o, double* out, void* stream);
+
+/* bsa_plan_heads: the head-wise compression plan of one layer and step
+ * (DiTFastAttnV2, "efficient compression plan search"): one method per head
+ * minimising the total latency subject to
+ *   I(h, m_h) <= c * delta / H   for every head (c = 1.5 in the pages), and
+ *   sum_h I(h, m_h) <= delta.
+ * Exact: a dynamic program over the integer total cost. Host only (no GPU).
+ *  rse: host double [H * M], rse[h * M + m] = I(h, m) (from bsa_rse).
+ *  cost: host int64 [H * M], >= 0, the latency of method m on head h in any
+ *    integer unit (the number of computed blocks for the attention modes).
+ *  choice: host int32 [H] out, the chosen method per head. Among plans of
+ *    equal cost the one with the least total error is returned.
+ *  total_cost: host int64 out, may be NULL.
+ *  Uses host memory proportional to H * (sum over heads of the largest cost).
+ *  Errors: INVALID_ARG (null pointer, H or M < 1, negative cost, delta or c
+ *  negative or not finite, total cost above 2^31), INFEASIBLE. */
+int bsa_plan_heads(int32_t H, int32_t M, const double* rse, const int64_t* cost, double delta, double c,
+                   int32_t* choice, int64_t* total_cost);
 
 /* Synchronise `stream`, then read and clear the device error word.
  * *code receives a BSA_DEVERR_* value. Returns BSA_OK, or BSA_ERR_CUDA if the
