@@ -22,12 +22,13 @@ HEAD_FULL, HEAD_SPARSE, HEAD_SKIP = 0, 1, 2
 BLOCK_NONE, BLOCK_FULL, BLOCK_PARTIAL = 0, 1, 2
 MASK_ARROW, MASK_GNA = 1, 2
 SELECT_POOLED_QK, SELECT_FULL_SCORE = 1, 2
+STEP_FULL, STEP_SELECT, STEP_REUSE = 0, 1, 2
 
 EXPORTS = (
     "bsa_version", "bsa_error_string", "bsa_build_mask", "bsa_select_workspace_size",
     "bsa_select_topk", "bsa_forward", "bsa_gna_tiled_len", "bsa_permute_tiles",
     "bsa_unpermute_tiles", "bsa_get_device_error", "bsa_select_topk_static", "bsa_rse",
-    "bsa_plan_heads",
+    "bsa_plan_heads", "bsa_schedule_full_steps", "bsa_step_action", "bsa_keep_pct", "bsa_jaccard",
 )
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -108,6 +109,11 @@ def _lib():
         lib.bsa_rse.argtypes = [P, P, P, P, P]
         lib.bsa_plan_heads.argtypes = [ctypes.c_int32, ctypes.c_int32, P, P, ctypes.c_double, ctypes.c_double,
                                        P, P]
+        I32 = ctypes.c_int32
+        lib.bsa_schedule_full_steps.argtypes = [I32, I32, P]
+        lib.bsa_step_action.argtypes = [I32, I32, I32, P]
+        lib.bsa_keep_pct.argtypes = [I32, I32, I32, I32, I32, I32, P]
+        lib.bsa_jaccard.argtypes = [P, P, P, P, P]
         _LIB = lib
     return _LIB
 
@@ -280,6 +286,34 @@ def plan_heads(rse_hm, cost_hm, delta: float, c: float = 1.5):
                                  float(delta), float(c), choice.ctypes.data_as(ctypes.c_void_p),
                                  ctypes.byref(total)), "bsa_plan_heads")
     return choice, int(total.value)
+
+
+def schedule_full_steps(n_steps: int, skip_pct: int) -> int:
+    """bsa_schedule_full_steps (host only)."""
+    v = ctypes.c_int32(0)
+    _check(_lib().bsa_schedule_full_steps(n_steps, skip_pct, ctypes.byref(v)), "bsa_schedule_full_steps")
+    return v.value
+
+
+def step_action(step: int, n_steps: int, n_full: int) -> int:
+    """bsa_step_action (host only): STEP_FULL, STEP_SELECT or STEP_REUSE."""
+    v = ctypes.c_int32(0)
+    _check(_lib().bsa_step_action(step, n_steps, n_full, ctypes.byref(v)), "bsa_step_action")
+    return v.value
+
+
+def keep_pct(layer: int, n_layers: int, step: int, n_steps: int, hi: int, lo: int) -> int:
+    """bsa_keep_pct (host only)."""
+    v = ctypes.c_int32(0)
+    _check(_lib().bsa_keep_pct(layer, n_layers, step, n_steps, hi, lo, ctypes.byref(v)), "bsa_keep_pct")
+    return v.value
+
+
+def jaccard(dm: Dims, a: BlockList, b: BlockList, out, stream=None):
+    """bsa_jaccard: out (cuda float32 [B, H, nQB]) receives the per-row similarity."""
+    ca, cb = a.c(), b.c()
+    _check(_lib().bsa_jaccard(ctypes.byref(dm), ctypes.byref(ca), ctypes.byref(cb), _ptr(out, torch.float32, "out"),
+                              _stream(stream)), "bsa_jaccard")
 
 
 def get_device_error(stream=None) -> int:

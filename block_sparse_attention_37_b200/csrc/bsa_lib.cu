@@ -8,3 +8,4 @@
 #include "select.cu"
 #include "select_static.cu"
 #include "plan.cu"
+#include "schedule.cu"

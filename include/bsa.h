@@ -59,6 +59,11 @@ extern "C" {
 #define BSA_MASK_ARROW 1
 #define BSA_MASK_GNA 2
 
+/* ---- denoising-step actions (bsa_step_action) ------------------------- */
+#define BSA_STEP_FULL 0    /* full attention, no pattern yet              */
+#define BSA_STEP_SELECT 1  /* select the head-specific pattern, then sparse */
+#define BSA_STEP_REUSE 2   /* sparse with the pattern selected earlier    */
+
 #define BSA_SELECT_POOLED_QK 1    /* mean-pooled Q/K block scores              */
 #define BSA_SELECT_FULL_SCORE 2   /* avg-pooled softmax map (SparseD)          */
 
@@ -257,6 +262,40 @@ int bsa_rse(const bsa_dims* dims, const void* y_m, const void* y_o, double* out,
  *  negative or not finite, total cost above 2^31), INFEASIBLE. */
 int bsa_plan_heads(int32_t H, int32_t M, const double* rse, const int64_t* cost, double delta, double c,
                    int32_t* choice, int64_t* total_cost);
+
+/* Step schedule of the sparse path (SparseD, "overall framework": the first
+ * T x skip% denoising steps run full attention, the head-specific pattern is
+ * selected once at that step and reused by every later step; the GNA
+ * article's image results split 9 full steps of 28 the same way). Host only.
+ *  bsa_schedule_full_steps: *n_full = ceil(n_steps * skip_pct / 100).
+ *  bsa_step_action: *action = BSA_STEP_FULL for step < n_full,
+ *    BSA_STEP_SELECT at step == n_full, BSA_STEP_REUSE after.
+ *  Errors: INVALID_ARG (null output, n_steps < 1, step outside
+ *  [0, n_steps), n_full outside [0, n_steps], skip_pct outside [0, 100]). */
+int bsa_schedule_full_steps(int32_t n_steps, int32_t skip_pct, int32_t* n_full);
+int bsa_step_action(int32_t step, int32_t n_steps, int32_t n_full, int32_t* action);
+
+/* bsa_keep_pct: the kept-block percentage of a layer and denoising step
+ * (lmnt.cn BSA post, section 3.3: shallow layers and early steps keep more,
+ * about 30%, deep layers and late steps fewer, 10-15%; no formula is given).
+ * Reading: hi - (hi - lo) * (layer / (n_layers - 1) + step / (n_steps - 1)) / 2,
+ * a fraction being 0 when its count is 1, rounded to the nearest integer,
+ * halves up; exact integer arithmetic. Host only.
+ *  Errors: INVALID_ARG (null output, counts < 1, indices out of range,
+ *  percentages outside [0, 100]). */
+int bsa_keep_pct(int32_t layer, int32_t n_layers, int32_t step, int32_t n_steps, int32_t hi, int32_t lo,
+                 int32_t* pct);
+
+/* bsa_jaccard: how stable a selection is across steps (SparseD, "sparse
+ * reuse"): per (b, h, query block) row, |A n B| / |A u B| of the kept KV
+ * block sets of two block lists (two empty rows score 1).
+ *  dims: B, H, N and block_q give the rows (B * H * ceil(N / block_q)).
+ *  a, b: block lists with ascending rows (as bsa_build_mask and
+ *    bsa_select_topk write them); cnt and idx are read.
+ *  out: device float [B, H, nQB], caller-owned, overwritten.
+ *  A count outside [0, max_k] records BSA_DEVERR_BAD_INDEX (clamped).
+ *  Errors: INVALID_ARG, CUDA. */
+int bsa_jaccard(const bsa_dims* dims, const bsa_block_list* a, const bsa_block_list* b, float* out, void* stream);
 
 /* Synchronise `stream`, then read and clear the device error word.
  * *code receives a BSA_DEVERR_* value. Returns BSA_OK, or BSA_ERR_CUDA if the
