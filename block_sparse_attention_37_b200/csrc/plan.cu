@@ -110,8 +110,10 @@ extern "C" int bsa_plan_heads(int32_t H, int32_t M, const double* rse, const int
       if (cost[(size_t)h * M + m] > mx) mx = cost[(size_t)h * M + m];
     }
     max_total += mx;
-    if (max_total > (1ll << 31)) return BSA_ERR_INVALID_ARG;
   }
+  // the tables hold H * (max_total + 1) choices: keep them within 2^28
+  // entries (costs in coarse units, such as blocks, stay far below)
+  if ((long long)H * (max_total + 1) > (1ll << 28)) return BSA_ERR_UNSUPPORTED;
   const size_t W = (size_t)max_total + 1;
   const double inf = INFINITY;
   std::vector<double> best(W, inf), next(W);

@@ -259,7 +259,8 @@ int bsa_rse(const bsa_dims* dims, const void* y_m, const void* y_o, double* out,
  *  total_cost: host int64 out, may be NULL.
  *  Uses host memory proportional to H * (sum over heads of the largest cost).
  *  Errors: INVALID_ARG (null pointer, H or M < 1, negative cost, delta or c
- *  negative or not finite, total cost above 2^31), INFEASIBLE. */
+ *  negative or not finite), UNSUPPORTED (H * (that sum + 1) above 2^28:
+ *  express costs in coarser units), INFEASIBLE. */
 int bsa_plan_heads(int32_t H, int32_t M, const double* rse, const int64_t* cost, double delta, double c,
                    int32_t* choice, int64_t* total_cost);
 

@@ -68,6 +68,9 @@ def test_plan_infeasible_and_bad_arguments():
     with pytest.raises(bsa.BsaError) as e:
         bsa.plan_heads(np.array([[0.0]]), np.array([[1]]), float("nan"), 1.5)
     assert e.value.status == bsa.ERR_INVALID_ARG
+    with pytest.raises(bsa.BsaError) as e:  # tables too large: coarser cost units needed
+        bsa.plan_heads(np.zeros((4, 2)), np.array([[1 << 27, 0]] * 4), 0.1, 1.5)
+    assert e.value.status == bsa.ERR_UNSUPPORTED
 
 
 def test_plan_at_c2_scale_is_feasible_and_locally_optimal():
