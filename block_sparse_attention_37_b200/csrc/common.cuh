@@ -163,53 +163,16 @@ __device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t a_desc, uint64
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem], A read from tensor memory
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                        uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same two MMA forms with the per-k-step offsets as compile-time
-// immediates added inside the asm (descriptor offsets in 16-byte units,
-// tensor-memory offsets in columns). Recomputing full 64-bit descriptors in
-// C++ before every instruction measured ~200 cycles per MMA from one issuing
-// thread; a loop-invariant base plus an immediate issues at the tensor core's
-// rate (~64 cycles for 128x128x16).
-template <uint32_t OFFA, uint32_t OFFB>
-__device__ __forceinline__ void umma_ss_at(uint32_t d_tmem, uint64_t a_base, uint64_t b_base, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 da, db;\n\t"
-      "add.s64 da, %1, %5;\n\t"
-      "add.s64 db, %2, %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], da, db, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_base), "l"(b_base), "r"(idesc), "r"(accumulate), "n"(OFFA), "n"(OFFB)
-      : "memory");
-}
-
-template <uint32_t OFFT, uint32_t OFFB>
-__device__ __forceinline__ void umma_ts_at(uint32_t d_tmem, uint32_t a_tmem_base, uint64_t b_base, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b32 ta;\n\t.reg .b64 db;\n\t"
-      "add.u32 ta, %1, %5;\n\t"
-      "add.s64 db, %2, %6;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [ta], db, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem_base), "l"(b_base), "r"(idesc), "r"(accumulate), "n"(OFFT), "n"(OFFB)
-      : "memory");
-}
-
-// Warp-wide forms for an issuer loop run by all 32 lanes (its state stays
+// MMA forms for an issuer loop run by all 32 lanes (its state stays
 // warp-uniform): one elected lane issues the MMA or the commit. The whole
 // warp must be converged; the elected lane is always the same (the lowest),
-// so commits track that lane's MMAs.
+// so commits track that lane's MMAs. The per-k-step offsets are compile-time
+// immediates added inside the asm (descriptor offsets in 16-byte units,
+// tensor-memory offsets in columns): recomputing full 64-bit descriptors in
+// C++ before every instruction measured ~200 cycles per MMA from one issuing
+// thread, while a loop-invariant base plus an immediate issues at the tensor
+// core's rate (~64 cycles for 128x128x16). The second form reads A from
+// tensor memory.
 template <uint32_t OFFA, uint32_t OFFB>
 __device__ __forceinline__ void umma_ss_at_warp(uint32_t d_tmem, uint64_t a_base, uint64_t b_base, uint32_t idesc,
                                                 uint32_t accumulate) {

@@ -214,8 +214,9 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
 }
 
 // Work order of the grid (longest first, so no long CTA starts late): all
-// FULL heads, then the SPARSE heads (below), then the SKIP heads. A bijection from blockIdx.x onto the B*H*nQP (b, h, pair)
-// items; heads with an invalid mode count as sparse (their CTA reports it).
+// FULL heads, then the SPARSE heads (below), then the SKIP heads. A
+// bijection from blockIdx.x onto the B*H*nQP (b, h, pair) items; heads with
+// an invalid mode count as sparse (their CTA reports it).
 // Run by a whole warp; every warp computes the same answer.
 __device__ __forceinline__ void map_item(const AttnParams& p, int d, int nQP, int lane, int& bh, int& pair) {
   int nF = 0, nK = 0;
@@ -641,13 +642,12 @@ __global__ void __launch_bounds__(384, 1)
         }
       }
     } else {
-      // Fixed issue order with blocking (suspending) waits, per tile t:
-      // QK^T(t) of each warpgroup that needs t, then the PV of each such
-      // warpgroup's previous tile. With separate P columns QK^T(t) waits only
-      // for S to be read, so it overlaps the softmax of the previous tile; with
-      // P written over S the PV goes first. All 32 lanes run the loop, so its
-      // state and the operand descriptors are warp-uniform; one elected lane
-      // issues each MMA and commit.
+      // P written over S: fixed issue order with blocking (suspending) waits.
+      // Per tile t, for each warpgroup that needs t: the PV of its previous
+      // tile, then QK^T(t) (the tensor pipe keeps issue order, so S is
+      // overwritten only after P has been read). All 32 lanes run the loop,
+      // so its state and the operand descriptors are warp-uniform; one
+      // elected lane issues each MMA and commit.
       if (T > 0) {
         constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
@@ -684,12 +684,9 @@ __global__ void __launch_bounds__(384, 1)
             if (!wwait(&q_full[w], 0u)) return false;
             q = true;
           }
-          const int c = w ? c1 : c0;
-          if (C::SEP_P) {
-            if (c > 0 && !wwait(&s_free[w], (uint32_t)(c - 1) & 1u)) return false;
-          } else if ((w ? pt1 : pt0) >= 0 && !pv(w)) {
-            return false;
-          }
+          // P is written over S: the previous PV must be issued first (the
+          // tensor pipe keeps issue order)
+          if ((w ? pt1 : pt0) >= 0 && !pv(w)) return false;
           tc_fence_after();
           qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::TILE, 16, 1024),
                  smem_desc_sw128(sKa + (t % S) * C::TILE, 16, 1024), idesc_qk,
@@ -714,10 +711,6 @@ __global__ void __launch_bounds__(384, 1)
           const int nw = tile_need(sched, nseg, t, act);
           if (nw & 1) ok = qk(0, t);
           if (ok && (nw & 2)) ok = qk(1, t);
-          if (C::SEP_P) {
-            if (ok && (nw & 1) && pt0 >= 0) ok = pv(0);
-            if (ok && (nw & 2) && pt1 >= 0) ok = pv(1);
-          }
           if (nw & 1) {
             pt0 = t;
             pj0 = c0++;
