@@ -397,15 +397,20 @@ def time_steps(job, steps, warmup, flush, with_fwd_events=True):
     return step_ms, fwd_ms
 
 
+# the workloads whose forward the oracle sampler times (the arrow ones; the
+# others add selection or GNA steps it does not run)
+ORACLE_CONFIGS = ("c1", "c2")
+
+
 def oracle_sample_tflops(cfg, budget_s, seed=0):
     """Time the fp64 oracle on a bounded sample of the workload (host cores)."""
     from threadpoolctl import threadpool_info
 
     from oracle import attention as OA
     from oracle import masks as OM
+    if cfg not in ORACLE_CONFIGS:
+        raise ValueError(f"the oracle baseline covers {ORACLE_CONFIGS} only")
     w = CONFIGS[cfg][1](DEFAULT_SEEDS[cfg])
-    if cfg not in ("c1", "c2"):
-        w = W.c2(1)  # the oracle baseline is taken on the arrow workload
     s = w["shape"]
     rng = np.random.default_rng(seed)
     heads = [(b, h) for b in range(s.B) for h in range(s.H) if int(w["head_mode"][h]) != W.HEAD_SKIP]
@@ -430,7 +435,7 @@ def oracle_sample_tflops(cfg, budget_s, seed=0):
     el = time.perf_counter() - t0
     threads = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas") or 1
     return {"value": flops / el / 1e12, "unit": UNIT, "cores": int(threads), "kind": "oracle",
-            "sample": f"{done} of {len(heads)} computed (b,h) heads of the SD3-1024-like workload, all rows, "
+            "sample": f"{done} of {len(heads)} computed (b,h) heads of the {cfg} workload, all rows, "
                       f"{el:.1f} s wall", "seconds": el}
 
 
@@ -441,7 +446,12 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     cfg = args.config
-    desc = CONFIGS[cfg][0] if cfg in ("c1", "c2") else CONFIGS["c2"][0]
+    if cfg not in ORACLE_CONFIGS:
+        print(json.dumps({"impl": "reference",
+                          "unavailable": f"the oracle arm times the arrow workloads {ORACLE_CONFIGS} only"}),
+              flush=True)
+        return 0
+    desc = CONFIGS[cfg][0]
     per_step = max(0.2, min(3.0, 150.0 / max(1, args.steps + args.warmup)))
     for _ in range(args.warmup):
         oracle_sample_tflops(cfg, per_step * 0.2)
@@ -526,7 +536,7 @@ def run_bsa(args, rank, world, local_rank):
                "ms_per_step": e2e_ms}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and cfg in ORACLE_CONFIGS:
         cpu = oracle_sample_tflops(cfg, args.cpu_seconds)
         cpu.pop("seconds", None)
 
