@@ -10,6 +10,8 @@ Random interleavings are explored on the workloads' key schedules and on
 random ones. Checked:
 
 * no deadlock: some agent can always move until all are done;
+  (schedules: the SD3-1024-like arrow CTAs, C3-like pooled top-30% CTAs,
+  random ones with long per-warpgroup gaps)
 * no stale data: every QK^T / PV finds its own tile in the K / V stage it
   reads, no stage is reloaded while an issued MMA still reads it, and the
   softmax never overwrites P that a pending PV reads.
@@ -173,10 +175,14 @@ def run(need, S, sep_p, seed, plant=None, max_steps=400000):
 
     def issuer_fixed():  # P over S
         pt, pj, c, q = [-1, -1], [0, 0], [0, 0], [False, False]
+        v_seen = [0]
 
         def pv(w):
             u = pt[w]
-            yield from wait(lambda: bar(f'v_full{u % S}').test((u // S) & 1))
+            while v_seen[0] <= u:  # V tiles observed in tile order, as in the kernel
+                x = v_seen[0]
+                yield from wait(lambda x=x: bar(f'v_full{x % S}').test((x // S) & 1))
+                v_seen[0] += 1
             yield from wait(lambda: bar(f'p_full{w}', 1).test(pj[w] & 1))
             issue(w, 'pv', u, pj[w])
             pt[w] = -1
@@ -280,6 +286,30 @@ def arrow_needs(N=4352, n_text=256, bs=64, windows=(1, 2, 4)):
     return out
 
 
+def pooled_needs():
+    """C3-like schedules: content-driven top-30% at block 128 (a CTA's two
+    warpgroups serve different query blocks, so their kept sets differ)."""
+    import workloads as W
+    from oracle import select as OS
+    w = W.content_case(B=1, H=2, n_text=256, grid_hw=(64, 64), d=64, block=128, seed=5)
+    shp = w["shape"]
+    ntb = -(-shp.n_text // shp.block_k)
+    groups = [(ntb, shp.n_kb, (30 * (shp.n_kb - ntb) + 99) // 100)]
+    out = []
+    for h in range(shp.H):
+        cls, _ = OS.pooled_select(w["q"][0, h].double().numpy(), w["k"][0, h].double().numpy(), 128, 128,
+                                  shp.n_text, groups, True)
+        for I in range(0, shp.n_qb, 2):  # CTA rows: warpgroup 0 = block I, warpgroup 1 = block I + 1
+            need = []
+            for J in range(shp.n_kb):  # a 128-key tile is one block (two 64-key segments)
+                b0 = cls[I, J] > 0
+                b1 = I + 1 < shp.n_qb and cls[I + 1, J] > 0
+                if b0 or b1:
+                    need.append((1 if b0 else 0) | (2 if b1 else 0))
+            out.append(need)
+    return out
+
+
 def random_needs(seed, n=40):
     rng = random.Random(seed)
     out = []
@@ -298,6 +328,15 @@ def random_needs(seed, n=40):
 def test_protocol_on_arrow_schedules(sep_p, S):
     for need in arrow_needs():
         for seed in range(6):
+            assert run(need, S, sep_p, seed) == 'ok', need
+
+
+@pytest.mark.parametrize("sep_p,S", [(True, 4), (False, 2)])
+def test_protocol_on_pooled_selection_schedules(sep_p, S):
+    needs = pooled_needs()
+    assert any(0 < sum(1 for n in need if n != 3) for need in needs)  # the warpgroups' sets differ
+    for need in needs:
+        for seed in range(4):
             assert run(need, S, sep_p, seed) == 'ok', need
 
 
