@@ -76,6 +76,16 @@ def test_host_argument_checks_return_before_launch():
     g = bsa.GnaGeom.make((8,), (64,), (4,), (5,))
     n = ctypes.c_int32(0)
     assert lib.bsa_gna_tiled_len(0, ctypes.byref(g), ctypes.byref(n)) == bsa.ERR_INVALID_ARG
+    # bsa_rse: null output, unaligned input, N*d not a multiple of 8
+    assert lib.bsa_rse(ctypes.byref(dm), p, p, None, None) == bsa.ERR_INVALID_ARG
+    assert lib.bsa_rse(ctypes.byref(dm), bad, p, p, None) == bsa.ERR_INVALID_ARG
+    dm3 = bsa.dims(1, 1, 3, 4, 64, 64, 0)
+    assert lib.bsa_rse(ctypes.byref(dm3), p, p, p, None) == bsa.ERR_UNSUPPORTED
+    # bsa_jaccard: missing list or output
+    assert lib.bsa_jaccard(ctypes.byref(dm), ctypes.byref(lst2), None, p, None) == bsa.ERR_INVALID_ARG
+    assert lib.bsa_jaccard(ctypes.byref(dm), ctypes.byref(lst2), ctypes.byref(lst2), None, None) \
+        == bsa.ERR_INVALID_ARG
+    assert lib.bsa_error_string(bsa.ERR_INFEASIBLE) == b"no plan meets the error budget"
 
 
 @pytest.mark.parametrize("n_text,grid,tile", [(256, (16, 48, 80), (4, 8, 8)), (5, (3, 5, 6), (2, 2, 4)),
