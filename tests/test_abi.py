@@ -56,6 +56,10 @@ def test_host_argument_checks_return_before_launch():
     dm = bsa.dims(1, 1, 128, 64, 48, 64, 0)
     assert lib.bsa_forward(ctypes.byref(dm), p, p, p, None, mode, None, None, None, None, 1.0, p, None) \
         == bsa.ERR_UNSUPPORTED
+    # the key schedule holds 2048 segments of 64 keys: N = 131072 is the largest sequence
+    dm_max = bsa.dims(1, 1, 131073, 64, 64, 64, 0)
+    assert lib.bsa_forward(ctypes.byref(dm_max), p, p, p, None, mode, None, None, None, None, 1.0, p, None) \
+        == bsa.ERR_UNSUPPORTED
     bad = ctypes.c_void_p(257)  # not 16-byte aligned
     dm = bsa.dims(1, 1, 128, 64, 64, 64, 0)
     assert lib.bsa_forward(ctypes.byref(dm), bad, p, p, None, mode, None, None, None, None, 1.0, p, None) \
