@@ -128,18 +128,38 @@ def _check(status: int, where: str):
         raise BsaError(status, where)
 
 
-def _ptr(t, dtype=None, name="tensor"):
+def _check_buffer(t, dtype=None, name="tensor", numel=None):
+    """Type, dtype and size of `t` (None passes). The library reads and writes
+    through raw pointers, so a buffer smaller than the layout the header states
+    would be accessed out of bounds: refuse it here."""
     if t is None:
-        return None
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if numel is not None and t.numel() < numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; these dims need {numel}")
+
+
+def _ptr(t, dtype=None, name="tensor", numel=None):
+    """Device pointer of `t` after the buffer check and the device checks."""
+    if t is None:
+        return None
+    _check_buffer(t, dtype, name, numel)
     if not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device (the library has no CPU path)")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
-    if dtype is not None and t.dtype != dtype:
-        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _ptrs(*specs):
+    """Pointers for (tensor, dtype, name, numel) specs. Every type and size is
+    checked before any device check, so a wrong size is reported as such."""
+    for sp in specs:
+        _check_buffer(*sp)
+    return [_ptr(*sp) for sp in specs]
 
 
 def _stream(stream):
@@ -158,6 +178,18 @@ def dims(B, H, N, d, block_q, block_k, n_text) -> Dims:
 
 def n_blocks(n: int, bs: int) -> int:
     return -(-n // bs)
+
+
+def _tokens(dm: Dims) -> int:
+    """Elements of one [B, H, N, d] tensor."""
+    return max(dm.B, 0) * max(dm.H, 0) * max(dm.N, 0) * max(dm.d, 0)
+
+
+def _grid(dm: Dims):
+    """(rows, nQB, nKB) of the block lists and bitmaps for these dims."""
+    nQB = n_blocks(dm.N, dm.block_q) if dm.block_q > 0 else 0
+    nKB = n_blocks(dm.N, dm.block_k) if dm.block_k > 0 else 0
+    return max(dm.B, 0) * max(dm.H, 0) * nQB, nQB, nKB
 
 
 @dataclass
@@ -179,19 +211,28 @@ class BlockList:
             bitmap=torch.empty((B, H, nQB, nKB), dtype=torch.uint8, device=device) if bitmap else None,
             max_k=max_k)
 
-    def c(self) -> BlockListC:
-        return BlockListC(_ptr(self.cnt, torch.int32, "cnt"), _ptr(self.idx, torch.int32, "idx"),
-                          _ptr(self.flag, torch.uint8, "flag"),
-                          _ptr(self.bitmap, torch.uint8, "bitmap"), self.max_k)
+    def specs(self, dm: Dims | None = None):
+        """Buffer specs of cnt, idx, flag and bitmap; with `dm`, each must hold
+        its [B, H, nQB(, max_k | nKB)] layout."""
+        rows, _, nKB = _grid(dm) if dm is not None else (None, 0, 0)
+        need = (lambda w: rows * w) if dm is not None else (lambda w: None)
+        return [(self.cnt, torch.int32, "cnt", need(1)), (self.idx, torch.int32, "idx", need(self.max_k)),
+                (self.flag, torch.uint8, "flag", need(self.max_k)),
+                (self.bitmap, torch.uint8, "bitmap", need(nKB))]
+
+    def c(self, dm: Dims | None = None, ptrs=None) -> BlockListC:
+        """The C struct (from already checked pointers, if given)."""
+        p = _ptrs(*self.specs(dm)) if ptrs is None else ptrs
+        return BlockListC(*p, self.max_k)
 
 
 # ---------------------------------------------------------------------------- calls
 
 def build_mask(dm: Dims, kind: int, out: BlockList, head_mode=None, window=None, gna: GnaGeom | None = None,
                stream=None):
-    spec = MaskSpec(kind, _ptr(head_mode, torch.int32, "head_mode"), _ptr(window, torch.int32, "window"),
-                    gna if gna is not None else GnaGeom())
-    lc = out.c()
+    p = _ptrs(*out.specs(dm), (head_mode, torch.int32, "head_mode", dm.H), (window, torch.int32, "window", dm.H))
+    spec = MaskSpec(kind, p[4], p[5], gna if gna is not None else GnaGeom())
+    lc = out.c(dm, p[:4])
     _check(_lib().bsa_build_mask(ctypes.byref(dm), ctypes.byref(spec), ctypes.byref(lc), _stream(stream)),
            "bsa_build_mask")
 
@@ -212,32 +253,39 @@ def select_workspace_size(dm: Dims, spec: SelectSpec) -> int:
 
 
 def select_topk(dm: Dims, q, k, spec: SelectSpec, out: BlockList, workspace, bias=None, stream=None):
-    lc = out.c()
-    _check(_lib().bsa_select_topk(ctypes.byref(dm), _ptr(q, torch.bfloat16, "Q"), _ptr(k, torch.bfloat16, "K"),
-                                  ctypes.byref(spec), _ptr(bias, torch.float32, "bias"),
-                                  _ptr(workspace, None, "workspace"), workspace.numel() * workspace.element_size(),
+    n, (_, nQB, nKB) = _tokens(dm), _grid(dm)
+    p = _ptrs(*out.specs(dm), (q, torch.bfloat16, "Q", n), (k, torch.bfloat16, "K", n),
+              (bias, torch.float32, "bias", dm.H * nQB * nKB), (workspace, None, "workspace", None))
+    lc = out.c(dm, p[:4])
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(_lib().bsa_select_topk(ctypes.byref(dm), p[4], p[5], ctypes.byref(spec), p[6], p[7], ws_bytes,
                                   ctypes.byref(lc), _stream(stream)), "bsa_select_topk")
 
 
 def select_topk_static(dm: Dims, q, k, spec: SelectSpec, out: BlockList, bias=None, stream=None):
     """bsa_select_topk_static: selection with the library's fixed scratch (no allocation)."""
-    lc = out.c()
-    _check(_lib().bsa_select_topk_static(ctypes.byref(dm), _ptr(q, torch.bfloat16, "Q"),
-                                         _ptr(k, torch.bfloat16, "K"), ctypes.byref(spec),
-                                         _ptr(bias, torch.float32, "bias"), ctypes.byref(lc), _stream(stream)),
+    n, (_, nQB, nKB) = _tokens(dm), _grid(dm)
+    p = _ptrs(*out.specs(dm), (q, torch.bfloat16, "Q", n), (k, torch.bfloat16, "K", n),
+              (bias, torch.float32, "bias", dm.H * nQB * nKB))
+    lc = out.c(dm, p[:4])
+    _check(_lib().bsa_select_topk_static(ctypes.byref(dm), p[4], p[5], ctypes.byref(spec), p[6], ctypes.byref(lc),
+                                         _stream(stream)),
            "bsa_select_topk_static")
 
 
 def forward(dm: Dims, q, k, v, o, head_mode, blocks: BlockList | None = None, gna: GnaGeom | None = None,
             cache_in=None, cache_out=None, bias=None, scale: float | None = None, stream=None):
     scale = (1.0 / dm.d ** 0.5) if scale is None else scale
-    lc = blocks.c() if blocks is not None else None
-    _check(_lib().bsa_forward(ctypes.byref(dm), _ptr(q, torch.bfloat16, "Q"), _ptr(k, torch.bfloat16, "K"),
-                              _ptr(v, torch.bfloat16, "V"), ctypes.byref(lc) if lc is not None else None,
-                              _ptr(head_mode, torch.int32, "head_mode"),
-                              ctypes.byref(gna) if gna is not None else None,
-                              _ptr(cache_in, torch.float32, "cache_in"), _ptr(cache_out, torch.float32, "cache_out"),
-                              _ptr(bias, torch.float32, "bias"), float(scale), _ptr(o, torch.bfloat16, "O"),
+    n, (_, nQB, nKB) = _tokens(dm), _grid(dm)
+    ls = blocks.specs(dm) if blocks is not None else []
+    p = _ptrs(*ls, (q, torch.bfloat16, "Q", n), (k, torch.bfloat16, "K", n), (v, torch.bfloat16, "V", n),
+              (o, torch.bfloat16, "O", n), (head_mode, torch.int32, "head_mode", dm.H),
+              (cache_in, torch.float32, "cache_in", n), (cache_out, torch.float32, "cache_out", n),
+              (bias, torch.float32, "bias", dm.H * nQB * nKB))
+    lc = blocks.c(dm, p[:4]) if blocks is not None else None
+    qp, kp, vp, op, hm, ci, co, bp = p[len(ls):]
+    _check(_lib().bsa_forward(ctypes.byref(dm), qp, kp, vp, ctypes.byref(lc) if lc is not None else None, hm,
+                              ctypes.byref(gna) if gna is not None else None, ci, co, bp, float(scale), op,
                               _stream(stream)), "bsa_forward")
 
 
@@ -247,29 +295,48 @@ def gna_tiled_len(n_text: int, gna: GnaGeom) -> int:
     return int(n.value)
 
 
-def _ptr_array(ts, name):
-    arr = (ctypes.c_void_p * len(ts))()
-    for i, t in enumerate(ts):
-        arr[i] = _ptr(t, torch.bfloat16, f"{name}[{i}]").value
-    return arr
+def _ptr_arrays(ins, n_in, outs, n_out):
+    """Host arrays of the device pointers of `ins` and `outs` (bf16, checked)."""
+    if len(ins) != len(outs):
+        raise ValueError("the permutation needs as many outputs as inputs")
+    specs = [(t, torch.bfloat16, f"in[{i}]", n_in) for i, t in enumerate(ins)] + \
+            [(t, torch.bfloat16, f"out[{i}]", n_out) for i, t in enumerate(outs)]
+    p = _ptrs(*specs)
+    a_in, a_out = (ctypes.c_void_p * len(ins))(), (ctypes.c_void_p * len(outs))()
+    for i in range(len(ins)):
+        a_in[i], a_out[i] = p[i].value, p[len(ins) + i].value
+    return a_in, a_out
+
+
+def _permute_sizes(dm: Dims, gna: GnaGeom):
+    """Elements of one raster tensor and of one tile-order tensor."""
+    grid = 1
+    for i in range(max(0, min(gna.ndim, 3))):
+        grid *= gna.grid[i]
+    bhd = max(dm.B, 0) * max(dm.H, 0) * max(dm.d, 0)
+    return bhd * (dm.n_text + grid), bhd * gna_tiled_len(dm.n_text, gna)
 
 
 def permute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
-    _check(_lib().bsa_permute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), _ptr_array(ins, "in"),
-                                    _ptr_array(outs, "out"), _stream(stream)), "bsa_permute_tiles")
+    n_r, n_t = _permute_sizes(dm, gna)
+    a_in, a_out = _ptr_arrays(ins, n_r, outs, n_t)
+    _check(_lib().bsa_permute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), a_in, a_out, _stream(stream)),
+           "bsa_permute_tiles")
 
 
 def unpermute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
-    _check(_lib().bsa_unpermute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), _ptr_array(ins, "in"),
-                                      _ptr_array(outs, "out"), _stream(stream)), "bsa_unpermute_tiles")
+    n_r, n_t = _permute_sizes(dm, gna)
+    a_in, a_out = _ptr_arrays(ins, n_t, outs, n_r)
+    _check(_lib().bsa_unpermute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), a_in, a_out, _stream(stream)),
+           "bsa_unpermute_tiles")
 
 
 def rse(dm: Dims, y_m, y_o, out, stream=None):
     """bsa_rse: out (cuda float64 [4*H]) receives I(h) then the three sums per head."""
-    if out.dtype != torch.float64 or not out.is_cuda or out.numel() < 4 * dm.H:
-        raise ValueError("out must be a cuda float64 tensor of 4*H elements")
-    _check(_lib().bsa_rse(ctypes.byref(dm), _ptr(y_m, torch.bfloat16, "y_m"), _ptr(y_o, torch.bfloat16, "y_o"),
-                          ctypes.c_void_p(out.data_ptr()), _stream(stream)), "bsa_rse")
+    n = _tokens(dm)
+    p = _ptrs((y_m, torch.bfloat16, "y_m", n), (y_o, torch.bfloat16, "y_o", n),
+              (out, torch.float64, "out", 4 * max(dm.H, 0)))
+    _check(_lib().bsa_rse(ctypes.byref(dm), *p, _stream(stream)), "bsa_rse")
 
 
 def plan_heads(rse_hm, cost_hm, delta: float, c: float = 1.5):
@@ -311,9 +378,10 @@ def keep_pct(layer: int, n_layers: int, step: int, n_steps: int, hi: int, lo: in
 
 def jaccard(dm: Dims, a: BlockList, b: BlockList, out, stream=None):
     """bsa_jaccard: out (cuda float32 [B, H, nQB]) receives the per-row similarity."""
-    ca, cb = a.c(), b.c()
-    _check(_lib().bsa_jaccard(ctypes.byref(dm), ctypes.byref(ca), ctypes.byref(cb), _ptr(out, torch.float32, "out"),
-                              _stream(stream)), "bsa_jaccard")
+    p = _ptrs(*a.specs(dm), *b.specs(dm), (out, torch.float32, "out", _grid(dm)[0]))
+    ca, cb = a.c(dm, p[0:4]), b.c(dm, p[4:8])
+    _check(_lib().bsa_jaccard(ctypes.byref(dm), ctypes.byref(ca), ctypes.byref(cb), p[8], _stream(stream)),
+           "bsa_jaccard")
 
 
 def get_device_error(stream=None) -> int:
