@@ -248,6 +248,12 @@ class ContentJob(Job):
         self.blocks_computed = self.blocks_total if dense else int(self.blocks.cnt.to(torch.int64).sum())
         self.flops = 4.0 * s.block_q * s.block_k * s.d * self.blocks_computed
 
+    def phases(self):
+        """The HBM-bound steps, each with its algorithmic bytes: pooling reads Q and K once."""
+        bsa, s = self.bsa, self.s
+        return [("select", lambda: bsa.select_topk(self.dm, self.q, self.k, self.spec, self.blocks, self.ws),
+                 select_bytes(s.B, s.H, s.N, s.d))]
+
     def step(self, ev_fwd=None):
         bsa = self.bsa
         bsa.select_topk(self.dm, self.q, self.k, self.spec, self.blocks, self.ws)
@@ -325,6 +331,14 @@ class VideoJob(Job):
         self.blocks_computed = int(self.blocks.cnt.to(torch.int64).sum())
         self.flops = 4.0 * s.block_q * s.block_k * s.d * self.blocks_computed
 
+    def phases(self):
+        """The HBM-bound steps, each with its algorithmic bytes (every row read once, written once)."""
+        bsa, s, nt = self.bsa, self.dm_r, self.dm.N
+        return [("permute", lambda: bsa.permute_tiles(self.dm_r, self.geom, self.raster, self.tiled),
+                 permute_bytes(s.B, s.H, s.N, nt, s.d, 3)),
+                ("unpermute", lambda: bsa.unpermute_tiles(self.dm_r, self.geom, [self.o_t], [self.o]),
+                 unpermute_bytes(s.B, s.H, s.N, s.d, 1))]
+
     def step(self, ev_fwd=None):
         bsa = self.bsa
         bsa.permute_tiles(self.dm_r, self.geom, self.raster, self.tiled)
@@ -374,6 +388,44 @@ def reduce_max(vals, world: int, device) -> list:
 def job_throughput(flops_per_step: float, world: int, ms_per_step: float) -> float:
     """Whole-job TFLOP/s: the units all ranks processed over the slowest rank's time."""
     return flops_per_step * world / (ms_per_step * 1e-3) / 1e12
+
+
+# ----------------------------------------------------------------------------- HBM-bound phases
+
+def select_bytes(B, H, N, d):
+    """Pooled selection: Q and K (bf16) read once; the pooled means and scores stay in L2."""
+    return 2 * B * H * N * d * 2
+
+
+def permute_bytes(B, H, n_raster, n_tiled, d, n_tensors):
+    """Raster -> tile order: every raster row read, every tile-order row (padding too) written."""
+    return n_tensors * B * H * (n_raster + n_tiled) * d * 2
+
+
+def unpermute_bytes(B, H, n_raster, d, n_tensors):
+    """Tile order -> raster: the real rows read and written; padding rows are dropped."""
+    return n_tensors * B * H * 2 * n_raster * d * 2
+
+
+def phase_bandwidth(phases, flush, hbm_gbs, reps=20, warmup=3):
+    """Each phase timed alone (CUDA events, L2 flushed before every call, median of `reps`),
+    as GB/s of its algorithmic bytes against the measured HBM copy bandwidth."""
+    out = {}
+    for name, fn, nbytes in phases:
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        ms = float(np.median([e0.elapsed_time(e1) for e0, e1 in evs]))
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "algorithmic_bytes": int(nbytes), "gbs": gbs, "frac_of_hbm": gbs / hbm_gbs}
+    return out
 
 
 # ----------------------------------------------------------------------------- timing
@@ -516,6 +568,10 @@ def run_bsa(args, rank, world, local_rank):
         del dense
     if isinstance(job, DlmJob):
         extra["selection_ms"] = job.selection_ms
+    if hasattr(job, "phases"):
+        hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+        extra["hbm_phases"] = phase_bandwidth(job.phases(), flush, hbm)
+        extra["hbm_peak_gbs"] = f"{hbm} ({peak_src} copy bandwidth)"
 
     e2e = None
     if not args.no_e2e and hasattr(job, "e2e_setup"):

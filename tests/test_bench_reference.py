@@ -33,3 +33,47 @@ def test_reference_line_on_c1():
 def test_reference_is_unavailable_where_the_oracle_does_not_time():
     d = _run("--config", "c4", "--steps", "1", "--warmup", "0")
     assert d["impl"] == "reference" and "unavailable" in d
+
+
+def test_hbm_phase_bytes_match_the_stated_traffic():
+    import bench
+    # pooled selection at the FLUX-2048-like size reads Q and K once: 2 x 103.8 MB
+    assert bench.select_bytes(1, 24, 16896, 128) == 2 * 24 * 16896 * 128 * 2
+    assert abs(bench.select_bytes(1, 24, 16896, 128) / 1e6 - 207.6) < 0.1
+    # the video workload (256 text + 16x48x80, no padding): the forward permute of Q, K, V and
+    # the inverse of O together move about 3.03 GB
+    n = 256 + 16 * 48 * 80
+    fw = bench.permute_bytes(1, 24, n, n, 128, 3)
+    bw = bench.unpermute_bytes(1, 24, n, 128, 1)
+    assert fw == 3 * 24 * 2 * n * 128 * 2 and bw == 24 * 2 * n * 128 * 2
+    assert abs((fw + bw) / 1e9 - 3.03) < 0.01
+    # padding rows are written by the forward permute but not read back by the inverse
+    assert bench.permute_bytes(1, 1, 100, 128, 8, 1) == (100 + 128) * 8 * 2
+    assert bench.unpermute_bytes(1, 1, 100, 8, 1) == 2 * 100 * 8 * 2
+
+
+def test_phase_bandwidth_reports_median_and_fraction(monkeypatch):
+    import bench
+    import torch
+
+    class FakeEvent:  # stands in for torch.cuda.Event: successive pairs are 2 ms apart
+        t = 0.0
+
+        def __init__(self, enable_timing=True):
+            self.at = None
+
+        def record(self):
+            FakeEvent.t += 1.0
+            self.at = FakeEvent.t
+
+        def elapsed_time(self, other):
+            return 2.0
+    monkeypatch.setattr(torch.cuda, "Event", FakeEvent)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    calls = []
+    out = bench.phase_bandwidth([("p", lambda: calls.append(1), 13_102_800)], torch.zeros(4), 6551.4, reps=5,
+                                warmup=2)
+    assert len(calls) == 7
+    p = out["p"]
+    assert p["ms"] == 2.0 and p["algorithmic_bytes"] == 13_102_800
+    assert abs(p["gbs"] - 6.5514) < 1e-9 and abs(p["frac_of_hbm"] - 0.001) < 1e-12
