@@ -330,6 +330,7 @@ class VideoJob(Job):
         self.blocks_total = s.B * s.H * nb * nb
         self.blocks_computed = int(self.blocks.cnt.to(torch.int64).sum())
         self.flops = 4.0 * s.block_q * s.block_k * s.d * self.blocks_computed
+        self.useful_flops = 4.0 * s.d * s.B * s.H * gna_useful_pairs(s.n_text, g.grid, g.window)
 
     def phases(self):
         """The HBM-bound steps, each with its algorithmic bytes (every row read once, written once)."""
@@ -405,6 +406,17 @@ def permute_bytes(B, H, n_raster, n_tiled, d, n_tensors):
 def unpermute_bytes(B, H, n_raster, d, n_tensors):
     """Tile order -> raster: the real rows read and written; padding rows are dropped."""
     return n_tensors * B * H * 2 * n_raster * d * 2
+
+
+def gna_useful_pairs(n_text, grid, window):
+    """Allowed (query, key) pairs of one head under the GNA mask: a video query sees exactly the
+    product of its per-dimension window lengths (the window is clamped inside the grid) plus the
+    text; a text query sees every real token. Padding is neither query nor key."""
+    n_img, win = 1, 1
+    for L, k in zip(grid, window):
+        n_img *= L
+        win *= min(k, L)
+    return n_img * (win + n_text) + n_text * (n_text + n_img)
 
 
 def phase_bandwidth(phases, flush, hbm_gbs, reps=20, warmup=3):
@@ -568,6 +580,9 @@ def run_bsa(args, rank, world, local_rank):
         del dense
     if isinstance(job, DlmJob):
         extra["selection_ms"] = job.selection_ms
+    if hasattr(job, "useful_flops"):  # pairs the mask allows, partial tiles counted by their real pairs
+        extra["useful_tflops"] = job.useful_flops / (fwd_ms_mean * 1e-3) / 1e12
+        extra["useful_flops_per_step"] = job.useful_flops
     if hasattr(job, "phases"):
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         extra["hbm_phases"] = phase_bandwidth(job.phases(), flush, hbm)
@@ -612,6 +627,8 @@ def run_bsa(args, rank, world, local_rank):
                    "l2": "flushed before every step (256 MiB write), flush outside the timed events",
                    "parallelism": f"independent replica per GPU x{world}", "seed": DEFAULT_SEEDS[cfg]},
         "pct_of_bf16_peak": 100.0 * value / world / peak,
+        "pct_of_bf16_sustained": 100.0 * value / world
+        / peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,

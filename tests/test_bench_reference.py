@@ -77,3 +77,16 @@ def test_phase_bandwidth_reports_median_and_fraction(monkeypatch):
     p = out["p"]
     assert p["ms"] == 2.0 and p["algorithmic_bytes"] == 13_102_800
     assert abs(p["gbs"] - 6.5514) < 1e-9 and abs(p["frac_of_hbm"] - 0.001) < 1e-12
+
+
+def test_gna_useful_pairs_equal_the_token_mask():
+    import bench
+    from oracle import masks as OM
+    cases = [(5, (3, 5, 6), (2, 2, 4), (2, 3, 3), (1, 1, 1)), (0, (7, 9), (4, 4), (3, 4), (1, 2)),
+             (3, (10,), (4,), (4,), (2,)), (17, (4, 6, 10), (2, 4, 8), (4, 4, 8), (2, 4, 8)),
+             (9, (6, 6), (4, 4), (6, 6), (3, 3))]
+    for n_text, grid, tile, window, stride in cases:
+        lay = OM.GnaLayout(n_text, grid, tile, window, stride)
+        assert int(OM.gna_token_mask(lay).sum()) == bench.gna_useful_pairs(n_text, grid, window), grid
+    # the video workload: 61,440 video queries x (3,072 + 256) keys + 256 text rows x 61,696
+    assert 4 * 128 * 24 * bench.gna_useful_pairs(256, (16, 48, 80), (8, 16, 24)) == 2_706_634_702_848
