@@ -68,3 +68,31 @@ def test_fp8_forward_is_the_plain_forward_on_representable_inputs():
     a = OA.head_forward(*deq, 0, fn, d ** -0.5)
     b = OA.head_forward(q, k, vv, 0, fn, d ** -0.5)
     np.testing.assert_array_equal(a, b)
+
+
+def test_encoding_matches_torch_float8_bytes():
+    # every finite value, both zeros included, against PyTorch's float8_e4m3fn bit patterns
+    v = np.concatenate([OF8.e4m3_values(), [-0.0]])
+    ref = torch.from_numpy(v.astype(np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(OF8.encode_e4m3(v), ref)
+    assert OF8.encode_e4m3([448.0, 2.0 ** -9, 1.0]).tolist() == [0x7E, 0x01, 0x38]
+    with pytest.raises(ValueError):
+        OF8.encode_e4m3([1.03])
+
+
+def test_fp32_decision_agrees_with_the_definition():
+    rng = np.random.default_rng(4)
+    x = (rng.normal(0, 1, (640, 128)) * rng.choice([1e-3, 1.0, 50.0], (640, 1))).astype(np.float32)
+    c32, s32 = OF8.quantize_fp32(x)
+    c64, s64 = OF8.quantize(x.astype(np.float64))
+    np.testing.assert_allclose(s32, s64, rtol=2 ** -23)   # fl32(amax / 448) vs the exact ratio
+    same = c32 == c64
+    assert same.mean() > 0.9999
+    # where they differ, they are neighbouring e4m3 values (a boundary straddled by fp32 rounding)
+    vals = OF8.e4m3_values()
+    idx = lambda a: np.searchsorted(vals, a)
+    assert np.all(np.abs(idx(c32[~same]) - idx(c64[~same])) == 1)
+    # every block's largest magnitude still lands on +-448, and zero blocks keep scale 1
+    for b in range(10):
+        assert np.abs(c32[b * 64:(b + 1) * 64]).max() == 448.0
+    assert np.all(OF8.quantize_fp32(np.zeros((64, 8)))[1] == 1.0)
