@@ -8,9 +8,31 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "../../include/bsa.h"
 
 namespace bsa {
+
+// ---------------------------------------------------------------------------
+// One-time setup of a kernel on each device (function attributes are per
+// device): a bit per device, set once the setup has succeeded there. Two
+// threads making the first call together both run the setup, which is
+// idempotent.
+struct DeviceOnce {
+  std::atomic<unsigned long long> done{0ull};
+  template <class F>
+  cudaError_t run(F&& setup) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = setup();
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+  }
+};
 
 // ---------------------------------------------------------------------------
 // device error word: first fault wins; read and cleared by bsa_get_device_error

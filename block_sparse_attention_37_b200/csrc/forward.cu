@@ -923,18 +923,17 @@ template <int D>
 static cudaError_t launch_fwd_d(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
   auto fn = fwd_kernel<D>;
-  static bool configured = false;
-  if (!configured) {
+  static DeviceOnce once;
+  const cudaError_t e = once.run([&]() -> cudaError_t {
     // the register split needs the full launch allocation: a smaller one
     // would leave setmaxnreg.inc waiting, so refuse to launch instead
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, fn);
-    if (e != cudaSuccess) return e;
+    cudaError_t r = cudaFuncGetAttributes(&fa, fn);
+    if (r != cudaSuccess) return r;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM_ALLOC);
+  });
+  if (e != cudaSuccess) return e;
   fn<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM_ALLOC, stream>>>(q, k, v, o, p);
   return cudaGetLastError();
 }

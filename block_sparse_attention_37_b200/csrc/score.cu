@@ -230,12 +230,11 @@ template <int D, int KIND>
 static cudaError_t launch_score_d(const CUtensorMap& q, const CUtensorMap& k, const AttnParams& p, int grid,
                                   cudaStream_t stream) {
   auto fn = score_kernel<D, KIND>;
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreCfg<D>::SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static DeviceOnce once;
+  const cudaError_t e = once.run([&]() -> cudaError_t {
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, ScoreCfg<D>::SMEM_ALLOC);
+  });
+  if (e != cudaSuccess) return e;
   fn<<<grid, 192, ScoreCfg<D>::SMEM_ALLOC, stream>>>(q, k, p);
   return cudaGetLastError();
 }
