@@ -9,7 +9,7 @@
 namespace bsa {
 
 // Raster row feeding tile-order position `pos`, or -1 for a padding slot.
-__device__ __forceinline__ int tile_source_row(const GnaDev& g, int pos) {
+__host__ __device__ __forceinline__ int tile_source_row(const GnaDev& g, int pos) {
   if (pos < g.n_text) return pos;
   if (pos < g.text_span) return -1;
   const int v = pos - g.text_span;

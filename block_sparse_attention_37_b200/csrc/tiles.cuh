@@ -26,7 +26,7 @@ __device__ __forceinline__ uint32_t bit_range(int a, int b) {  // bits [a, b), c
   return hi & ~lo;
 }
 
-__device__ __forceinline__ uint64_t bit_range64(int a, int b) {  // bits [a, b), clipped to [0, 64)
+__host__ __device__ __forceinline__ uint64_t bit_range64(int a, int b) {  // bits [a, b), clipped to [0, 64)
   a = max(a, 0);
   b = min(b, 64);
   if (a >= b) return 0ull;
@@ -58,7 +58,7 @@ struct QWin {
   int lo0, lo1, lo2, hi0, hi1, hi2;
 };
 
-__device__ __forceinline__ QWin gna_query_window(const GnaDev& g, int pq, bool windowed) {
+__host__ __device__ __forceinline__ QWin gna_query_window(const GnaDev& g, int pq, bool windowed) {
   QWin w{0, 0, 0, 1 << 30, 1 << 30, 1 << 30};
   if (!windowed || pq < g.text_span) return w;
   const int v = pq - g.text_span;
@@ -78,7 +78,7 @@ __device__ __forceinline__ QWin gna_query_window(const GnaDev& g, int pq, bool w
 
 // Allowed-key bits of one 64-key segment (tile order) for a query window.
 // Needs the tile's x-extent to divide 64 or be a multiple of 64.
-__device__ __forceinline__ uint64_t gna_segment_bits(const GnaDev& g, int seg, const QWin& q) {
+__host__ __device__ __forceinline__ uint64_t gna_segment_bits(const GnaDev& g, int seg, const QWin& q) {
   const int k0 = seg * 64;
   if (k0 < g.text_span) {
     const int nt = g.n_text - k0;

@@ -1,0 +1,111 @@
+"""The kernels' GNA index arithmetic, compiled for the host from the library's own
+sources, against the oracle (no GPU).
+
+The forward's fine mask of a PARTIAL tile (gna_query_window + gna_segment_bits)
+and the permutation's row map (tile_source_row) are host-callable functions of
+csrc/. A small harness that includes the library's single translation unit
+exposes them; every bit and every row index must equal what the oracle's
+token-level GNA mask and tile order give.
+"""
+import ctypes
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+from oracle import masks as OM
+from oracle import permute as OP
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "block_sparse_attention_37_b200", "csrc")
+
+HARNESS = r'''
+#include "bsa_lib.cu"
+extern "C" int h_segbits_row(int n_text, const bsa_gna_geom* geom, int pq, unsigned long long* out, int nseg) {
+  bsa::GnaDev g;
+  const int st = bsa::make_gna(geom, n_text, &g);
+  if (st) return st;
+  const bsa::QWin q = bsa::gna_query_window(g, pq, true);
+  for (int s = 0; s < nseg; ++s) out[s] = bsa::gna_segment_bits(g, s, q);
+  return 0;
+}
+extern "C" int h_tile_sources(int n_text, const bsa_gna_geom* geom, int* out, int n) {
+  bsa::GnaDev g;
+  const int st = bsa::make_gna(geom, n_text, &g);
+  if (st) return st;
+  for (int pos = 0; pos < n; ++pos) out[pos] = bsa::tile_source_row(g, pos);
+  return 0;
+}
+'''
+
+
+@pytest.fixture(scope="module")
+def host_lib(tmp_path_factory):
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not found: the harness is compiled from the library's CUDA sources")
+    d = tmp_path_factory.mktemp("host_index_math")
+    src = d / "harness.cu"
+    src.write_text(HARNESS)
+    so = d / "harness.so"
+    cmd = [nvcc, "-O2", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-Xcompiler", "-fPIC",
+           "-shared", "-I", os.path.join(ROOT, "include"), "-I", CSRC, "-o", str(so), str(src)]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lib = ctypes.CDLL(str(so))
+    lib.h_segbits_row.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
+    lib.h_tile_sources.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    return lib
+
+
+class Geom(ctypes.Structure):  # bsa_gna_geom
+    _fields_ = [("ndim", ctypes.c_int32), ("grid", ctypes.c_int32 * 3), ("tile", ctypes.c_int32 * 3),
+                ("window", ctypes.c_int32 * 3), ("stride", ctypes.c_int32 * 3)]
+
+
+def _geom(grid, tile, window, stride):
+    g = Geom()
+    g.ndim = len(grid)
+    for i in range(len(grid)):
+        g.grid[i], g.tile[i], g.window[i], g.stride[i] = grid[i], tile[i], window[i], stride[i]
+    return g
+
+
+CASES = [
+    (64, (4, 8, 16), (2, 4, 8), (3, 5, 7), (1, 1, 1)),        # partial tiles everywhere
+    (50, (5, 9, 20), (2, 4, 8), (3, 5, 7), (1, 2, 2)),        # padding in the grid and the text
+    (0, (300,), (64,), (97,), (5,)),                            # 1-D, padded last tile
+    (128, (8, 256), (1, 128), (3, 48), (1, 16)),                # tile x extent wider than a segment
+    (17, (6, 10, 12), (2, 2, 16), (4, 5, 6), (2, 1, 3)),        # mixed strides, ragged text
+    (256, (16, 48, 80), (4, 8, 8), (8, 16, 24), (1, 1, 1)),     # the video workload, stride 1
+    (256, (16, 48, 80), (4, 8, 8), (8, 16, 24), (4, 8, 8)),     # the video workload, stride 4x8x8
+]
+
+
+@pytest.mark.parametrize("n_text,grid,tile,window,stride", CASES)
+def test_fine_mask_bits_equal_the_token_mask(host_lib, n_text, grid, tile, window, stride):
+    lay = OM.GnaLayout(n_text, grid, tile, window, stride)
+    g = _geom(grid, tile, window, stride)
+    nseg = -(-lay.N // 64)
+    rows = np.arange(lay.N)
+    if lay.N > 4096:
+        rows = np.sort(np.random.default_rng(lay.N).choice(lay.N, 256, replace=False))
+    rows = rows[lay.valid(rows)]
+    out = np.zeros(nseg, dtype=np.uint64)
+    shifts = np.arange(64, dtype=np.uint64)
+    for pq in rows:
+        assert host_lib.h_segbits_row(n_text, ctypes.byref(g), int(pq), out.ctypes.data, nseg) == 0
+        got = ((out[:, None] >> shifts[None, :]) & np.uint64(1)).astype(bool).reshape(-1)[:lay.N]
+        exp = OM.gna_token_mask(lay, [int(pq)])[0]
+        assert np.array_equal(got, exp), (grid, int(pq), np.nonzero(got != exp)[0][:5])
+
+
+@pytest.mark.parametrize("n_text,grid,tile,window,stride", CASES)
+def test_permutation_row_map_equals_the_tile_order(host_lib, n_text, grid, tile, window, stride):
+    lay = OM.GnaLayout(n_text, grid, tile, window, stride)
+    g = _geom(grid, tile, window, stride)
+    out = np.empty(lay.N, dtype=np.int32)
+    assert host_lib.h_tile_sources(n_text, ctypes.byref(g), out.ctypes.data, lay.N) == 0
+    np.testing.assert_array_equal(out, OP.tile_order_source(lay))
