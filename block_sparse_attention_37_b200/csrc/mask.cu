@@ -7,7 +7,7 @@
 namespace bsa {
 
 // Sum over queries i in [q_lo, q_hi) of |[start(i), start(i)+k) intersect [k_lo, k_hi)|.
-__device__ __forceinline__ long long pair_count_1d(int q_lo, int q_hi, int k_lo, int k_hi, int L,
+__host__ __device__ __forceinline__ long long pair_count_1d(int q_lo, int q_hi, int k_lo, int k_hi, int L,
                                                    int k, int s) {
   long long c = 0;
   for (int i = q_lo; i < q_hi; ++i) {
@@ -19,7 +19,7 @@ __device__ __forceinline__ long long pair_count_1d(int q_lo, int q_hi, int k_lo,
 }
 
 // Does KV block J hold padded (invalid) key slots?
-__device__ bool gna_kv_padded(const GnaDev& g, int J) {
+__host__ __device__ bool gna_kv_padded(const GnaDev& g, int J) {
   const int ntb = g.text_span / g.vol;
   if (J < ntb) return g.text_span > g.n_text && (J + 1) * g.vol > g.n_text;
   const int tile = J - ntb;
@@ -32,7 +32,7 @@ __device__ bool gna_kv_padded(const GnaDev& g, int J) {
 
 // Class of (query tile I, KV tile J) under the GNA window; text rows and
 // columns are full, padded key slots make a block partial.
-__device__ int gna_class(const GnaDev& g, int I, int J) {
+__host__ __device__ int gna_class(const GnaDev& g, int I, int J) {
   const int ntb = g.text_span / g.vol;
   const bool kpad = gna_kv_padded(g, J);
   if (I < ntb || J < ntb) return kpad ? BSA_BLOCK_PARTIAL : BSA_BLOCK_FULL;

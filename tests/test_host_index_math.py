@@ -1,11 +1,12 @@
 """The kernels' GNA index arithmetic, compiled for the host from the library's own
 sources, against the oracle (no GPU).
 
-The forward's fine mask of a PARTIAL tile (gna_query_window + gna_segment_bits)
-and the permutation's row map (tile_source_row) are host-callable functions of
-csrc/. A small harness that includes the library's single translation unit
-exposes them; every bit and every row index must equal what the oracle's
-token-level GNA mask and tile order give.
+The forward's fine mask of a PARTIAL tile (gna_query_window + gna_segment_bits),
+the mask builder's tile classes (gna_class) and the permutation's row map
+(tile_source_row) are host-callable functions of csrc/. A small harness that
+includes the library's single translation unit exposes them; every bit, class
+and row index must equal what the oracle's token-level GNA mask, its block
+classes and its tile order give.
 """
 import ctypes
 import os
@@ -29,6 +30,14 @@ extern "C" int h_segbits_row(int n_text, const bsa_gna_geom* geom, int pq, unsig
   if (st) return st;
   const bsa::QWin q = bsa::gna_query_window(g, pq, true);
   for (int s = 0; s < nseg; ++s) out[s] = bsa::gna_segment_bits(g, s, q);
+  return 0;
+}
+extern "C" int h_gna_classes(int n_text, const bsa_gna_geom* geom, unsigned char* out, int nb) {
+  bsa::GnaDev g;
+  const int st = bsa::make_gna(geom, n_text, &g);
+  if (st) return st;
+  for (int I = 0; I < nb; ++I)
+    for (int J = 0; J < nb; ++J) out[I * nb + J] = (unsigned char)bsa::gna_class(g, I, J);
   return 0;
 }
 extern "C" int h_tile_sources(int n_text, const bsa_gna_geom* geom, int* out, int n) {
@@ -57,6 +66,7 @@ def host_lib(tmp_path_factory):
     lib = ctypes.CDLL(str(so))
     lib.h_segbits_row.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
     lib.h_tile_sources.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    lib.h_gna_classes.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return lib
 
 
@@ -109,3 +119,19 @@ def test_permutation_row_map_equals_the_tile_order(host_lib, n_text, grid, tile,
     out = np.empty(lay.N, dtype=np.int32)
     assert host_lib.h_tile_sources(n_text, ctypes.byref(g), out.ctypes.data, lay.N) == 0
     np.testing.assert_array_equal(out, OP.tile_order_source(lay))
+
+
+@pytest.mark.parametrize("n_text,grid,tile,window,stride", CASES)
+def test_tile_classes_equal_the_oracle(host_lib, n_text, grid, tile, window, stride):
+    lay = OM.GnaLayout(n_text, grid, tile, window, stride)
+    g = _geom(grid, tile, window, stride)
+    nb = lay.N // lay.bs
+    out = np.empty(nb * nb, dtype=np.uint8)
+    assert host_lib.h_gna_classes(n_text, ctypes.byref(g), out.ctypes.data, nb) == 0
+    got = out.reshape(nb, nb)
+    if lay.N <= 4096:  # against the classes counted from the token-level mask
+        valid = lay.valid(np.arange(lay.N))
+        exp = OM.classify_blocks(OM.gna_token_mask(lay), lay.bs, lay.bs, valid, valid)
+    else:              # the separable counts (pinned to token enumeration on small layouts)
+        exp = OM.gna_block_classes_separable(lay)
+    np.testing.assert_array_equal(got, exp)
