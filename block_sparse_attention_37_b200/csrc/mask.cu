@@ -8,7 +8,7 @@ namespace bsa {
 
 // Sum over queries i in [q_lo, q_hi) of |[start(i), start(i)+k) intersect [k_lo, k_hi)|.
 __host__ __device__ __forceinline__ long long pair_count_1d(int q_lo, int q_hi, int k_lo, int k_hi, int L,
-                                                   int k, int s) {
+                                                            int k, int s) {
   long long c = 0;
   for (int i = q_lo; i < q_hi; ++i) {
     const int st = gna_window_start(i, L, k, s);
