@@ -169,14 +169,17 @@ def _stream(stream):
 
 
 def version() -> int:
+    """Library version, major*10000 + minor*100 + patch (bsa_version)."""
     return _lib().bsa_version()
 
 
 def dims(B, H, N, d, block_q, block_k, n_text) -> Dims:
+    """Problem shape (bsa_dims): batch, heads, tokens, head dim, query / key block sizes, text tokens."""
     return Dims(B, H, N, d, block_q, block_k, n_text)
 
 
 def n_blocks(n: int, bs: int) -> int:
+    """ceil(n / bs): blocks of size bs over n tokens (the last one ragged)."""
     return -(-n // bs)
 
 
@@ -230,6 +233,9 @@ class BlockList:
 
 def build_mask(dm: Dims, kind: int, out: BlockList, head_mode=None, window=None, gna: GnaGeom | None = None,
                stream=None):
+    """bsa_build_mask: arrow (MASK_ARROW, window per head in blocks) or GNA (MASK_GNA, tile-order
+    tokens, block = tile volume) block lists into `out` for every (b, h, query block).
+    head_mode / window: cuda int32 [H] (head_mode None = all SPARSE)."""
     p = _ptrs(*out.specs(dm), (head_mode, torch.int32, "head_mode", dm.H), (window, torch.int32, "window", dm.H))
     spec = MaskSpec(kind, p[4], p[5], gna if gna is not None else GnaGeom())
     lc = out.c(dm, p[:4])
@@ -238,6 +244,8 @@ def build_mask(dm: Dims, kind: int, out: BlockList, head_mode=None, window=None,
 
 
 def select_spec(method: int, groups, keep_text: bool, scale: float = 1.0) -> SelectSpec:
+    """Selection spec: method (SELECT_POOLED_QK / SELECT_FULL_SCORE), up to four (begin, end, k) key
+    block groups each cut to its own top k, whether text blocks are always kept, the logit scale."""
     sp = SelectSpec()
     sp.method = method
     sp.n_groups = len(groups)
@@ -249,10 +257,14 @@ def select_spec(method: int, groups, keep_text: bool, scale: float = 1.0) -> Sel
 
 
 def select_workspace_size(dm: Dims, spec: SelectSpec) -> int:
+    """Bytes of device workspace bsa_select_topk needs for these dims and spec."""
     return int(_lib().bsa_select_workspace_size(ctypes.byref(dm), ctypes.byref(spec)))
 
 
 def select_topk(dm: Dims, q, k, spec: SelectSpec, out: BlockList, workspace, bias=None, stream=None):
+    """bsa_select_topk: content-driven block lists into `out`. q, k: cuda bf16 [B, H, N, d];
+    workspace: cuda tensor of at least select_workspace_size bytes, 256-byte aligned;
+    bias: cuda fp32 [H, nQB, nKB] logit offset (FULL_SCORE) or None."""
     n, (_, nQB, nKB) = _tokens(dm), _grid(dm)
     p = _ptrs(*out.specs(dm), (q, torch.bfloat16, "Q", n), (k, torch.bfloat16, "K", n),
               (bias, torch.float32, "bias", dm.H * nQB * nKB), (workspace, None, "workspace", None))
@@ -275,6 +287,10 @@ def select_topk_static(dm: Dims, q, k, spec: SelectSpec, out: BlockList, bias=No
 
 def forward(dm: Dims, q, k, v, o, head_mode, blocks: BlockList | None = None, gna: GnaGeom | None = None,
             cache_in=None, cache_out=None, bias=None, scale: float | None = None, stream=None):
+    """bsa_forward: o (cuda bf16 [B, H, N, d]) = block-sparse attention of q, k, v (same shape) over
+    the kept blocks; per head FULL / SPARSE (the block list) / SKIP (o = bf16 of cache_in, fp32
+    [B, H, N, d]). cache_out receives the fp32 output of computed heads; bias is a cuda fp32
+    [H, nQB, nKB] logit offset; scale defaults to 1/sqrt(d); gna is needed for PARTIAL blocks."""
     scale = (1.0 / dm.d ** 0.5) if scale is None else scale
     n, (_, nQB, nKB) = _tokens(dm), _grid(dm)
     ls = blocks.specs(dm) if blocks is not None else []
@@ -290,6 +306,7 @@ def forward(dm: Dims, q, k, v, o, head_mode, blocks: BlockList | None = None, gn
 
 
 def gna_tiled_len(n_text: int, gna: GnaGeom) -> int:
+    """Tokens in tile order: text padded to a tile-volume multiple plus every (padded) tile."""
     n = ctypes.c_int32(0)
     _check(_lib().bsa_gna_tiled_len(int(n_text), ctypes.byref(gna), ctypes.byref(n)), "bsa_gna_tiled_len")
     return int(n.value)
@@ -318,6 +335,8 @@ def _permute_sizes(dm: Dims, gna: GnaGeom):
 
 
 def permute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
+    """bsa_permute_tiles: raster [B, H, n_text + prod(grid), d] bf16 tensors to tile order
+    [B, H, gna_tiled_len, d] (padding rows zeroed), one output per input (at most four)."""
     n_r, n_t = _permute_sizes(dm, gna)
     a_in, a_out = _ptr_arrays(ins, n_r, outs, n_t)
     _check(_lib().bsa_permute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), a_in, a_out, _stream(stream)),
@@ -325,6 +344,7 @@ def permute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
 
 
 def unpermute_tiles(dm: Dims, gna: GnaGeom, ins, outs, stream=None):
+    """bsa_unpermute_tiles: the inverse of permute_tiles (padding rows dropped)."""
     n_r, n_t = _permute_sizes(dm, gna)
     a_in, a_out = _ptr_arrays(ins, n_t, outs, n_r)
     _check(_lib().bsa_unpermute_tiles(ctypes.byref(dm), ctypes.byref(gna), len(ins), a_in, a_out, _stream(stream)),
@@ -385,6 +405,7 @@ def jaccard(dm: Dims, a: BlockList, b: BlockList, out, stream=None):
 
 
 def get_device_error(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device error word (a DEVERR_* value)."""
     code = ctypes.c_int32(0)
     _check(_lib().bsa_get_device_error(_stream(stream), ctypes.byref(code)), "bsa_get_device_error")
     return int(code.value)
