@@ -272,3 +272,16 @@ def test_forward_c4_sampled_rows_with_gpu_selection():
         exp = OA.head_forward(f64(q1[0, h]), f64(k1[0, h]), f64(v1[0, h]), 1, fn, 128 ** -0.5, rows=rows,
                               bias_fn=bfn)
         assert_close_out(f64(o[0, h])[rows], exp, f"c4 h{h}")
+
+
+@pytest.mark.slow
+def test_forward_at_the_schedule_capacity():
+    """N = 131072 tokens, the most a CTA's key schedule holds (2048 segments of 64 keys): one full
+    head and one arrow head; sampled rows, the first and the last included, against the oracle."""
+    w = W.arrow_case(B=1, H=2, n_text=256, grid_hw=(1, 131072 - 256), d=64, block=64, seed=13,
+                     fracs=(0.5, 0.5, 0.0), with_cache=False)
+    shp = w["shape"]
+    assert shp.N == 131072 and sorted(int(x) for x in w["head_mode"]) == [W.HEAD_FULL, W.HEAD_SPARSE]
+    o, _ = _run_arrow(w)
+    rows = np.unique(np.concatenate([[0, shp.N - 1], np.random.default_rng(13).choice(shp.N, 22, replace=False)]))
+    _check_arrow(w, o, rows=rows)
