@@ -86,6 +86,11 @@ int make_gna(const bsa_gna_geom* in, int n_text, GnaDev* g) {
   g->text_span = ceil_div(n_text, vol) * (int)vol;
   long long n_tiled = (long long)g->text_span + ntiles * vol;
   if (n_tiled > (1ll << 30)) return BSA_ERR_UNSUPPORTED;
+  g->f_vol = make_fastdiv(g->vol);
+  g->f_tiles2 = make_fastdiv(g->tiles[2]);
+  g->f_tiles1 = make_fastdiv(g->tiles[1]);
+  g->f_tile2 = make_fastdiv(g->tile[2]);
+  g->f_tile1 = make_fastdiv(g->tile[1]);
   g->has_padding = g->text_span > n_text;
   for (int d = 0; d < 3; ++d) g->has_padding |= (g->grid[d] % g->tile[d]) != 0;
   return BSA_OK;
@@ -129,6 +134,32 @@ SelectLayout select_layout(const bsa_dims* dm, const bsa_select_spec* sp) {
     L.total = L.apool + align256(BH * nQB * nKB * sizeof(float));
   }
   return L;
+}
+
+// Every argument check of bsa_select_topk except the workspace's, in the
+// order that call makes them. bsa_select_topk_static runs it before its own
+// scratch-size check, so both entry points report the same status for the
+// same unsupported or invalid request.
+int check_select_args(const bsa_dims* dims, const void* Q, const void* K, const bsa_select_spec* spec,
+                      const bsa_block_list* out) {
+  int st = check_dims(dims);
+  if (st != BSA_OK) return st;
+  if (!spec || !Q || !K || !aligned16(Q) || !aligned16(K)) return BSA_ERR_INVALID_ARG;
+  if (dims->d != 64 && dims->d != 128) return BSA_ERR_UNSUPPORTED;
+  const int nKB = ceil_div(dims->N, dims->block_k);
+  if ((st = check_list(out, nKB)) != BSA_OK) return st;
+  if (spec->n_groups < 0 || spec->n_groups > 4) return BSA_ERR_INVALID_ARG;
+  for (int g = 0; g < spec->n_groups; ++g) {
+    const bsa_key_group& kg = spec->groups[g];
+    if (kg.begin < 0 || kg.end > nKB || kg.begin > kg.end || kg.k < 0) return BSA_ERR_INVALID_ARG;
+  }
+  if (spec->method != BSA_SELECT_POOLED_QK && spec->method != BSA_SELECT_FULL_SCORE) return BSA_ERR_INVALID_ARG;
+  if ((size_t)nKB * 5 > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+  if (spec->method == BSA_SELECT_FULL_SCORE) {
+    if (dims->block_q != dims->block_k || dims->block_q % 128 != 0) return BSA_ERR_UNSUPPORTED;
+    if (ceil_div(dims->N, 64) > kMaxSeg) return BSA_ERR_UNSUPPORTED;
+  }
+  return BSA_OK;
 }
 
 }  // namespace
@@ -207,19 +238,9 @@ size_t bsa_select_workspace_size(const bsa_dims* dims, const bsa_select_spec* sp
 int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K, const bsa_select_spec* spec,
                     const float* block_bias, void* workspace, size_t workspace_bytes, const bsa_block_list* out,
                     void* stream) {
-  int st = check_dims(dims);
+  int st = check_select_args(dims, Q, K, spec, out);
   if (st != BSA_OK) return st;
-  if (!spec || !Q || !K || !aligned16(Q) || !aligned16(K)) return BSA_ERR_INVALID_ARG;
-  if (dims->d != 64 && dims->d != 128) return BSA_ERR_UNSUPPORTED;
   const int nQB = ceil_div(dims->N, dims->block_q), nKB = ceil_div(dims->N, dims->block_k);
-  if ((st = check_list(out, nKB)) != BSA_OK) return st;
-  if (spec->n_groups < 0 || spec->n_groups > 4) return BSA_ERR_INVALID_ARG;
-  for (int g = 0; g < spec->n_groups; ++g) {
-    const bsa_key_group& kg = spec->groups[g];
-    if (kg.begin < 0 || kg.end > nKB || kg.begin > kg.end || kg.k < 0) return BSA_ERR_INVALID_ARG;
-  }
-  if (spec->method != BSA_SELECT_POOLED_QK && spec->method != BSA_SELECT_FULL_SCORE) return BSA_ERR_INVALID_ARG;
-  if ((size_t)nKB * 5 > 200 * 1024) return BSA_ERR_UNSUPPORTED;
   const SelectLayout L = select_layout(dims, spec);
   if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return BSA_ERR_WORKSPACE;
@@ -264,8 +285,6 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K, const bs
     sp.qbar = pp.qbar;
     sp.kbar = pp.kbar;
   } else {
-    if (dims->block_q != dims->block_k || dims->block_q % 128 != 0) return BSA_ERR_UNSUPPORTED;
-    if (ceil_div(dims->N, 64) > kMaxSeg) return BSA_ERR_UNSUPPORTED;
     const long long BH = (long long)dims->B * dims->H;
     CUtensorMap mq, mk;
     if ((st = make_map(&mq, Q, BH, dims->N, dims->d)) != BSA_OK) return st;

@@ -305,12 +305,44 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------------------
 // GNA geometry as the kernels see it (all dimensions padded to 3, outermost first)
 
+// Division of a dividend below 2^31 by an invariant d >= 1 as a multiply-high
+// and a shift (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", 1994, with N = 31): l = ceil(log2 d), m = floor(2^(31+l) / d)
+// + 1 < 2^32, and floor(n / d) = floor(n * m / 2^(31+l)) for 0 <= n < 2^31.
+struct FastDiv {
+  uint32_t m;
+  int s;  // l - 1; -1 for d = 1
+  int d;
+};
+
+inline FastDiv make_fastdiv(int d) {
+  FastDiv f{0u, -1, d};
+  if (d <= 1) return f;
+  int l = 0;
+  while ((1ll << l) < d) ++l;
+  f.m = (uint32_t)(((1ull << (31 + l)) / (unsigned long long)d) + 1ull);
+  f.s = l - 1;
+  return f;
+}
+
+__host__ __device__ __forceinline__ int fdiv(int n, const FastDiv& f) {
+  if (f.s < 0) return n;
+#ifdef __CUDA_ARCH__
+  return (int)(__umulhi((uint32_t)n, f.m) >> f.s);
+#else
+  return (int)((((unsigned long long)(uint32_t)n * f.m) >> 32) >> f.s);
+#endif
+}
+
 struct GnaDev {
   int n_text;      // text tokens
   int text_span;   // text padded to a multiple of the tile volume
   int vol;         // tile volume = block size
   int grid[3], tile[3], win[3], stride[3], tiles[3];
   int has_padding; // any padded slot in the layout
+  // invariant divisors of the fine mask: tile volume, tiles along x, tiles along y,
+  // tile x extent, tile y extent
+  FastDiv f_vol, f_tiles2, f_tiles1, f_tile2, f_tile1;
 };
 
 __host__ __device__ __forceinline__ int gna_window_start(int i, int L, int k, int s) {

@@ -817,33 +817,31 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float mu = (m == kNegInf) ? 0.f : m;
       const float oa = ba - mu, ob = bb - mu;
-      // PV(j-1) must be complete before O is rescaled, and (own P columns)
-      // before P_w is overwritten; O is rescaled once S is dead (fewer live
-      // registers), which is safe because PV(j) waits for p_full
+      // P = exp2(x - m), packed to bf16 in registers first: nothing here
+      // touches tensor memory, so the exps overlap the previous PV
+      float sum0 = 0.f, sum1 = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float o = i < 32 ? oa : ob;
+        float x0 = sv[2 * i], x1 = sv[2 * i + 1];
+        fma2(x0, x1, cscale, o);
+        x0 = fast_exp2(x0);
+        x1 = fast_exp2(x1);
+        add2(sum0, sum1, x0, x1);
+        pk[i] = pack_bf16x2(x0, x1);
+      }
+      l = l * alpha + (sum0 + sum1);
+      // PV(j-1) must be complete before P is written (own P columns at d = 64,
+      // over S at d = 128) and before O is rescaled; O is rescaled once S is
+      // dead (fewer live registers), which is safe because PV(j) waits for p_full
       if (j > 0) {
         ok = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
         if (!ok) break;
         tc_fence_after();
       }
-      // P = exp2(x - m) per 32-key chunk, packed to bf16 (over the scores
-      // when P shares S's columns: S is already in registers)
-      float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float o = c < 2 ? oa : ob;
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0 = sv[32 * c + 2 * i], x1 = sv[32 * c + 2 * i + 1];
-          fma2(x0, x1, cscale, o);
-          x0 = fast_exp2(x0);
-          x1 = fast_exp2(x1);
-          add2(sum0, sum1, x0, x1);
-          pk[i] = pack_bf16x2(x0, x1);
-        }
-        tmem_st16(ptm + 16 * c, pk);
-      }
-      l = l * alpha + (sum0 + sum1);
+      for (int c = 0; c < 4; ++c) tmem_st16(ptm + 16 * c, pk + 16 * c);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {

@@ -2,8 +2,9 @@
 // (jsqmd.com GNA article, section 2.2: a dedicated copy kernel replacing
 // permute().contiguous(), fused with padding). Every token row is d bf16
 // values contiguous in memory, so both directions move whole rows with
-// 16-byte vector loads and stores; one thread moves one 16-byte chunk and the
-// grid strides over (tensor, b*h, tile-order row, chunk).
+// 16-byte vector loads and stores. One warp owns one tile-order row: its
+// source row is mapped once, then the warp moves that row for every tensor
+// and (b, h), so the index arithmetic is paid once per row, not per chunk.
 #include "permute.cuh"
 
 namespace bsa {
@@ -22,35 +23,60 @@ __host__ __device__ __forceinline__ int tile_source_row(const GnaDev& g, int pos
   return g.n_text + (t * g.grid[1] + y) * g.grid[2] + x;
 }
 
+// Lanes cover (b*h, chunk) pairs: with cpr 16-byte chunks per row, 32 / cpr
+// rows of different heads sit side by side in the warp (d = 128: 2, d = 64:
+// 4), each a contiguous run of cpr chunks, and every lane keeps four loads in
+// flight (four heads apart).
 template <bool FORWARD>
-__global__ void __launch_bounds__(256) permute_kernel(PermuteParams p) {
-  const int chunks = p.d >> 3;  // 16-byte chunks per row
-  const long long per_tensor = (long long)p.BH * p.n_tiled * chunks;
-  const long long total = per_tensor * p.n_tensors;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
-       i += (long long)gridDim.x * blockDim.x) {
-    const int t = (int)(i / per_tensor);
-    long long rem = i - (long long)t * per_tensor;
-    const int c = (int)(rem % chunks);
-    rem /= chunks;
-    const int pos = (int)(rem % p.n_tiled);
-    const long long bh = rem / p.n_tiled;
-    const int src = tile_source_row(p.g, pos);
-    if (FORWARD) {
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (src >= 0) v = __ldg(reinterpret_cast<const uint4*>(p.in[t] + (bh * p.n_raster + src) * p.d) + c);
-      reinterpret_cast<uint4*>(p.out[t] + (bh * p.n_tiled + pos) * p.d)[c] = v;
-    } else if (src >= 0) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.in[t] + (bh * p.n_tiled + pos) * p.d) + c);
-      reinterpret_cast<uint4*>(p.out[t] + (bh * p.n_raster + src) * p.d)[c] = v;
+__global__ void __launch_bounds__(256, 4) permute_kernel(PermuteParams p) {
+  const int lane = threadIdx.x & 31;
+  const int cpr = p.d >> 3;                         // 16-byte chunks per row
+  const int nsub = cpr >= 32 ? 1 : 32 / cpr;        // heads side by side in one warp
+  const int sub = cpr >= 32 ? 0 : lane / cpr;       // this lane's head within them
+  const int c_first = cpr >= 32 ? lane : lane % cpr;
+  const int c_step = cpr >= 32 ? 32 : cpr;          // one pass when a row fits the warp
+  const bool on = sub < nsub;                       // lanes past nsub * cpr idle
+  const long long bh_step = 4ll * nsub;
+  const int wpb = blockDim.x >> 5;
+  const int n_warps = gridDim.x * wpb;
+  for (int pos = blockIdx.x * wpb + (threadIdx.x >> 5); pos < p.n_tiled; pos += n_warps) {
+    int src = lane == 0 ? tile_source_row(p.g, pos) : 0;
+    src = __shfl_sync(0xffffffffu, src, 0);
+    if ((!FORWARD && src < 0) || !on) continue;  // padding rows are dropped by the inverse
+    for (int t = 0; t < p.n_tensors; ++t) {
+      const uint4* __restrict__ in = reinterpret_cast<const uint4*>(p.in[t]);
+      uint4* __restrict__ out = reinterpret_cast<uint4*>(p.out[t]);
+      for (long long bh0 = sub; bh0 < p.BH; bh0 += bh_step) {
+        for (int c = c_first; c < cpr; c += c_step) {
+          uint4 v[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const long long bh = bh0 + (long long)u * nsub;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (bh < p.BH && src >= 0) {
+              const long long row = FORWARD ? bh * p.n_raster + src : bh * p.n_tiled + pos;
+              v[u] = __ldg(in + row * cpr + c);
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const long long bh = bh0 + (long long)u * nsub;
+            if (bh < p.BH) {
+              const long long row = FORWARD ? bh * p.n_tiled + pos : bh * p.n_raster + src;
+              out[row * cpr + c] = v[u];
+            }
+          }
+        }
+      }
     }
   }
 }
 
+// One warp per row, up to 4 blocks of 8 warps per SM (64 registers a thread,
+// no spills; 32 warps x 4 loads of 16 B per lane keep ~64 KB per SM in flight).
 cudaError_t launch_permute(bool forward, const PermuteParams& p, int num_sms, cudaStream_t stream) {
-  const long long total = (long long)p.BH * p.n_tiled * (p.d >> 3) * p.n_tensors;
-  long long blocks = (total + 255) / 256;
-  const long long cap = (long long)num_sms * 8;
+  long long blocks = ((long long)p.n_tiled + 7) / 8;
+  const long long cap = (long long)num_sms * 4;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   if (forward)

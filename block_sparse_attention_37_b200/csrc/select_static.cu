@@ -36,10 +36,12 @@ int scratch_for_current_device(void** out) {
 extern "C" int bsa_select_topk_static(const bsa_dims* dims, const void* Q, const void* K,
                                       const bsa_select_spec* spec, const float* block_bias,
                                       const bsa_block_list* out, void* stream) {
-  if (!dims || !spec) return BSA_ERR_INVALID_ARG;
-  const size_t need = bsa_select_workspace_size(dims, spec);
-  if (need == 0) return BSA_ERR_INVALID_ARG;
-  if (need > (size_t)BSA_STATIC_SCRATCH_BYTES) return BSA_ERR_WORKSPACE;
+  // The same argument checks as bsa_select_topk come first, so an invalid or
+  // unsupported request is reported as such even when it is also too large
+  // for the scratch.
+  const int arg = bsa::check_select_args(dims, Q, K, spec, out);
+  if (arg != BSA_OK) return arg;
+  if (bsa_select_workspace_size(dims, spec) > (size_t)BSA_STATIC_SCRATCH_BYTES) return BSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   const int st = bsa::scratch_for_current_device(&scratch);
   if (st != BSA_OK) return st;

@@ -27,8 +27,8 @@ __device__ __forceinline__ uint32_t bit_range(int a, int b) {  // bits [a, b), c
 }
 
 __host__ __device__ __forceinline__ uint64_t bit_range64(int a, int b) {  // bits [a, b), clipped to [0, 64)
-  a = max(a, 0);
-  b = min(b, 64);
+  a = a > 0 ? a : 0;
+  b = b < 64 ? b : 64;
   if (a >= b) return 0ull;
   const uint64_t hi = b >= 64 ? ~0ull : ((1ull << b) - 1ull);
   const uint64_t lo = (1ull << a) - 1ull;
@@ -77,7 +77,9 @@ __host__ __device__ __forceinline__ QWin gna_query_window(const GnaDev& g, int p
 }
 
 // Allowed-key bits of one 64-key segment (tile order) for a query window.
-// Needs the tile's x-extent to divide 64 or be a multiple of 64.
+// Needs the tile's x-extent to divide 64 or be a multiple of 64. The segment's
+// place in the tile grid takes five divisions by launch invariants (multiply-
+// high and shift); the rows of the segment step a (t, y) counter.
 __host__ __device__ __forceinline__ uint64_t gna_segment_bits(const GnaDev& g, int seg, const QWin& q) {
   const int k0 = seg * 64;
   if (k0 < g.text_span) {
@@ -85,31 +87,39 @@ __host__ __device__ __forceinline__ uint64_t gna_segment_bits(const GnaDev& g, i
     return nt <= 0 ? 0ull : (nt >= 64 ? ~0ull : ((1ull << nt) - 1ull));
   }
   const int v0 = k0 - g.text_span;
-  const int tile = v0 / g.vol;
+  const int tile = fdiv(v0, g.f_vol);
   const int l0 = v0 - tile * g.vol;
-  const int tx = tile % g.tiles[2];
-  const int ty = (tile / g.tiles[2]) % g.tiles[1];
-  const int tt = tile / (g.tiles[2] * g.tiles[1]);
+  const int q2 = fdiv(tile, g.f_tiles2);
+  const int tx = tile - q2 * g.tiles[2];
+  const int tt = fdiv(q2, g.f_tiles1);
+  const int ty = q2 - tt * g.tiles[1];
   const int bt = tt * g.tile[0], by = ty * g.tile[1], bx = tx * g.tile[2];
   const int Tx = g.tile[2], Ty = g.tile[1];
-  const int xlo = max(q.lo2, 0), xhi = min(q.hi2, g.grid[2]);
+  const int xlo = q.lo2 > 0 ? q.lo2 : 0;
+  const int xhi = q.hi2 < g.grid[2] ? q.hi2 : g.grid[2];
+  const int tlo = q.lo0, thi = q.hi0 < g.grid[0] ? q.hi0 : g.grid[0];
+  const int ylo = q.lo1, yhi = q.hi1 < g.grid[1] ? q.hi1 : g.grid[1];
   uint64_t m = 0ull;
   if (Tx <= 64) {
-    const int rows = 64 / Tx;
-    const int R0 = l0 / Tx;
+    const int rows = 64 / Tx;  // Tx divides 64 (host check)
+    const int R0 = fdiv(l0, g.f_tile2);
+    int tq = fdiv(R0, g.f_tile1);
+    int yq = R0 - tq * Ty;
     const uint64_t xb = bit_range64(xlo - bx, xhi - bx) & bit_range64(0, Tx);
     for (int rr = 0; rr < rows; ++rr) {
-      const int R = R0 + rr;
-      const int t = bt + R / Ty, y = by + R % Ty;
-      const bool ok = t >= q.lo0 && t < q.hi0 && t < g.grid[0] && y >= q.lo1 && y < q.hi1 && y < g.grid[1];
-      if (ok) m |= xb << (rr * Tx);
+      const int t = bt + tq, y = by + yq;
+      if (t >= tlo && t < thi && y >= ylo && y < yhi) m |= xb << (rr * Tx);
+      if (++yq == Ty) {
+        yq = 0;
+        ++tq;
+      }
     }
   } else {
-    const int R = l0 / Tx;
+    const int R = fdiv(l0, g.f_tile2);
     const int xo = bx + (l0 - R * Tx);
-    const int t = bt + R / Ty, y = by + R % Ty;
-    const bool ok = t >= q.lo0 && t < q.hi0 && t < g.grid[0] && y >= q.lo1 && y < q.hi1 && y < g.grid[1];
-    if (ok) m = bit_range64(xlo - xo, xhi - xo);
+    const int tq = fdiv(R, g.f_tile1);
+    const int t = bt + tq, y = by + (R - tq * Ty);
+    if (t >= tlo && t < thi && y >= ylo && y < yhi) m = bit_range64(xlo - xo, xhi - xo);
   }
   return m;
 }

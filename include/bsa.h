@@ -181,12 +181,17 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K,
  *  allocated: no cudaMalloc, no cudaFree, no allocating library call.
  *  The first call on a device looks up the array's device address
  *  (cudaGetSymbolAddress) with that device current; make that first call
- *  before any stream capture on the device.
+ *  before any stream capture on the device. The address is cached for the
+ *  life of the process: it is not valid across a device reset
+ *  (cudaDeviceReset or a primary-context reset), after which this entry
+ *  point must not be called again in the same process.
  *  All calls share the one array, which keeps the previous call's contents
  *  (the kernels clear what must start at zero). Calls whose kernels overlap on
  *  the GPU (e.g. on two streams) race on the scratch: serialise them.
- *  Errors: those of bsa_select_topk, and BSA_ERR_WORKSPACE when
- *  bsa_select_workspace_size(dims, spec) exceeds BSA_STATIC_SCRATCH_BYTES. */
+ *  Errors: bsa_select_topk's argument checks run first and give the same
+ *  INVALID_ARG / UNSUPPORTED status; then BSA_ERR_WORKSPACE when
+ *  bsa_select_workspace_size(dims, spec) exceeds BSA_STATIC_SCRATCH_BYTES;
+ *  then the CUDA errors of bsa_select_topk. */
 int bsa_select_topk_static(const bsa_dims* dims, const void* Q, const void* K,
                            const bsa_select_spec* spec, const float* block_bias,
                            const bsa_block_list* out, void* stream);

@@ -1,11 +1,15 @@
 """Shared helpers of the GPU parity tests: run the library, ask the oracle, compare."""
 from __future__ import annotations
 
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
 from oracle import attention as OA
 from oracle import masks as OM
+from oracle import select as OS
 
 MAX_ABS = 2e-2   # spec tolerance for bf16 outputs
 MEAN_ABS = 5e-3
@@ -86,3 +90,47 @@ def selection_matches(got_row: np.ndarray, scores: np.ndarray, groups, fixed_kee
             return False, amb_total
         rest[b:e] = False
     return (not rest.any()), amb_total
+
+
+def oracle_workers() -> int:
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def full_score_rows(q, k, scale, bq, bk, rows, bias=None):
+    """fp64 [len(rows), nKB]: the oracle's A' rows for the given query blocks of one (b, h).
+
+    The rows are independent, so they are spread over a thread pool (numpy releases the GIL in
+    its matmul and exp); each row is the oracle's own avgpool_attention_rows."""
+    rows = [int(I) for I in rows]
+    with ThreadPoolExecutor(oracle_workers()) as ex:
+        out = list(ex.map(lambda I: OS.avgpool_attention_rows(q, k, scale, bq, bk, I, bias), rows))
+    return np.stack(out)
+
+
+def check_full_score_rows(cls_bh, q, k, scale, bq, bk, groups, rows, bias=None):
+    """Every listed query-block row of a GPU full-score selection of one (b, h) agrees with the
+    oracle's A' outside near-ties. Returns the oracle's A' rows."""
+    ap = full_score_rows(q, k, scale, bq, bk, rows, bias)
+    nkb = cls_bh.shape[-1]
+    for r, I in enumerate(rows):
+        ok, _ = selection_matches(cls_bh[I] > 0, ap[r], groups, np.zeros(nkb, bool))
+        assert ok, f"query block {I}"
+    return ap
+
+
+def check_pooled_rows(cls_bh, q, k, bq, bk, n_text, groups, rows):
+    """Every listed query-block row of a GPU pooled selection of one (b, h) agrees with the
+    oracle's pooled scores (text rows full, text key blocks kept, groups cut outside near-ties)."""
+    sc = OS.pooled_scores(q, k, bq, bk)
+    ntq, ntk = -(-n_text // bq), -(-n_text // bk)
+    nkb = cls_bh.shape[-1]
+    for I in rows:
+        row = cls_bh[I] > 0
+        if I < ntq:
+            assert row.all(), f"text query block {I} must be full"
+            continue
+        fixed = np.zeros(nkb, bool)
+        fixed[:ntk] = True
+        assert row[:ntk].all(), f"query block {I} must keep the text key blocks"
+        ok, _ = selection_matches(row, sc[I], groups, fixed)
+        assert ok, f"query block {I}"

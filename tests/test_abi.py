@@ -76,6 +76,25 @@ def test_host_argument_checks_return_before_launch():
     sp = bsa.select_spec(bsa.SELECT_POOLED_QK, [(0, 2, 1)], False)
     assert lib.bsa_select_topk(ctypes.byref(dm), p, p, ctypes.byref(sp), None, p, 16, ctypes.byref(lst2), None) \
         == bsa.ERR_WORKSPACE
+    # the allocation-free selection runs the same argument checks before its scratch-size check:
+    # an unsupported request that is also too large for the scratch reports UNSUPPORTED
+    big_bad = bsa.dims(1, 64, 131072, 96, 128, 128, 0)
+    lst_big = bsa.BlockListC(p, p, p, None, 1024)
+    fs = bsa.select_spec(bsa.SELECT_FULL_SCORE, [(0, 1024, 8)], False, 0.1)
+    assert lib.bsa_select_topk_static(ctypes.byref(big_bad), p, p, ctypes.byref(fs), None,
+                                      ctypes.byref(lst_big), None) == bsa.ERR_UNSUPPORTED
+    big_bs64 = bsa.dims(1, 64, 131072, 128, 64, 64, 0)
+    lst_big64 = bsa.BlockListC(p, p, p, None, 2048)
+    fs64 = bsa.select_spec(bsa.SELECT_FULL_SCORE, [(0, 2048, 8)], False, 0.1)
+    assert lib.bsa_select_topk_static(ctypes.byref(big_bs64), p, p, ctypes.byref(fs64), None,
+                                      ctypes.byref(lst_big64), None) == bsa.ERR_UNSUPPORTED
+    assert lib.bsa_select_topk_static(ctypes.byref(big_bs64), bad, p, ctypes.byref(fs64), None,
+                                      ctypes.byref(lst_big64), None) == bsa.ERR_INVALID_ARG
+    # a valid request above the fixed scratch size is refused before any launch
+    big_ok = bsa.dims(1, 64, 131072, 128, 128, 128, 0)
+    assert bsa.select_workspace_size(big_ok, fs) > 16 << 20
+    assert lib.bsa_select_topk_static(ctypes.byref(big_ok), p, p, ctypes.byref(fs), None,
+                                      ctypes.byref(lst_big), None) == bsa.ERR_WORKSPACE
     # invalid GNA geometry (stride > window)
     g = bsa.GnaGeom.make((8,), (64,), (4,), (5,))
     n = ctypes.c_int32(0)

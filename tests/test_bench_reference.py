@@ -30,9 +30,34 @@ def test_reference_line_on_c1():
     assert "workload" in d["config"]
 
 
-def test_reference_is_unavailable_where_the_oracle_does_not_time():
-    d = _run("--config", "c4", "--steps", "1", "--warmup", "0")
-    assert d["impl"] == "reference" and "unavailable" in d
+def test_reference_line_on_the_video_workload():
+    """The default workload (GNA video, stride 1): the oracle on sampled query tiles."""
+    d = _run("--steps", "1", "--warmup", "0")
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert "stride 1x1x1" in d["config"]["workload"]
+    assert "query tiles" in d["cpu_baseline"]["sample"]
+
+
+def test_oracle_sampler_credits_computed_blocks():
+    """The sampled units credit exactly the computed-block FLOPs of their rows: summed over every
+    unit of a workload, the credits equal the workload's total (arrow heads; GNA query tiles)."""
+    import numpy as np
+
+    import bench
+    import workloads as W
+    from oracle import masks as OM
+    w = W.c1()
+    units = bench._oracle_plan("c1", w, np.random.default_rng(0))
+    total = sum(run() for run, _, _ in units)
+    s = w["shape"]
+    kept = int((OM.arrow_block_classes_all(s, w["head_mode"], w["window"]) > 0).sum())
+    assert total == 4.0 * s.block_q * s.block_k * s.d * kept
+    v = W.video_case(1, 1, 16, (4, 8, 8), (2, 4, 4), (3, 5, 5), (1, 1, 1), 64, 5)
+    units = bench._oracle_plan("c5f", v, np.random.default_rng(0))
+    lay = OM.GnaLayout(16, (4, 8, 8), (2, 4, 4), (3, 5, 5), (1, 1, 1))
+    cls = OM.gna_block_classes_separable(lay)
+    sampled = sum(run() for run, _, _ in units)
+    assert len(units) == 2 and 0 < sampled <= 4.0 * lay.bs * lay.bs * 64 * 2 * cls.shape[0]
 
 
 def test_hbm_phase_bytes_match_the_stated_traffic():

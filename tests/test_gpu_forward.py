@@ -8,7 +8,7 @@ from oracle import attention as OA
 from oracle import masks as OM
 from oracle import permute as OP
 from oracle import select as OS
-from parity_util import arrow_expected, assert_close_out, bsa, f64
+from parity_util import arrow_expected, assert_close_out, bsa, check_pooled_rows, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -158,8 +158,28 @@ def test_forward_selected_blocks_from_oracle_selection():
         assert_close_out(f64(o[0, h]), exp, f"h{h}")
 
 
-def _gna_forward(B, H, n_text, grid, tile, window, stride, d, seed, modes, rows_per_head=None):
-    """Raster inputs -> GPU permute -> mask -> forward -> unpermute; oracle on sampled rows."""
+def _tile_rows(lay, tiles):
+    """Tile-order positions of every token of the listed tiles (tile coordinates per dim; None is
+    the text tile)."""
+    out = []
+    for t in tiles:
+        if t is None:
+            out.append(np.arange(lay.text_span))
+            continue
+        lin = 0
+        for c, n in zip(t, lay.tiles):
+            assert 0 <= c < n
+            lin = lin * n + c
+        start = lay.text_span + lin * lay.vol
+        out.append(np.arange(start, start + lay.vol))
+    return np.concatenate(out)
+
+
+def _gna_forward(B, H, n_text, grid, tile, window, stride, d, seed, modes, rows_per_head=None,
+                 all_rows_tiles=(), all_rows_heads=()):
+    """Raster inputs -> GPU permute -> mask -> forward -> unpermute; oracle on sampled rows.
+
+    Heads in ``all_rows_heads`` also compare every row of the tiles in ``all_rows_tiles``."""
     m = bsa()
     wl = W.video_case(B, H, n_text, grid, tile, window, stride, d, seed)
     lay = OM.GnaLayout(n_text, grid, tile, window, stride)
@@ -189,6 +209,9 @@ def _gna_forward(B, H, n_text, grid, tile, window, stride, d, seed, modes, rows_
             qt, kt, vt = (OP.permute_to_tiles(f64(t[b, h]), lay) for t in (wl["q"], wl["k"], wl["v"]))
             cand = np.nonzero(valid)[0]
             rows = cand if rows_per_head is None else np.sort(rng.choice(cand, rows_per_head, replace=False))
+            if h in all_rows_heads and rows_per_head is not None:
+                extra = _tile_rows(lay, all_rows_tiles)
+                rows = np.unique(np.concatenate([rows, extra[valid[extra]]]))
             mode = int(modes[h])
             if mode == OM.HEAD_FULL:
                 fn = lambda r: valid[np.asarray(r)][:, None] & valid[None, :]
@@ -209,15 +232,25 @@ def test_forward_gna_small(n_text, grid, tile, window, stride):
     _gna_forward(1, 3, n_text, grid, tile, window, stride, 128, 7, modes=[1, 0, 1])
 
 
+# Tiles of the 4 x 6 x 10 tile grid of the video workload where windows clamp: two opposite
+# corners, a corner on the other diagonal, and one tile on a face of each dimension; None is the
+# text tile (full rows).
+C5_EDGE_TILES = ((0, 0, 0), (3, 5, 9), (3, 5, 0), (0, 2, 4), (2, 0, 5), (1, 4, 9), None)
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("stride", [(4, 8, 8), (1, 1, 1)])
 def test_forward_c5_sampled_rows(stride):
+    """24 sampled rows of every head, plus every row of the corner and face tiles on three heads."""
     _gna_forward(1, 24, 256, (16, 48, 80), (4, 8, 8), (8, 16, 24), stride, 128, 4, modes=[1] * 24,
-                 rows_per_head=24)
+                 rows_per_head=24, all_rows_tiles=C5_EDGE_TILES, all_rows_heads=(0, 11, 23))
 
 
 def test_forward_c3_sampled_rows_with_gpu_selection():
-    """FLUX-2048-like: GPU pooled selection, then the GPU forward; oracle on sampled rows."""
+    """FLUX-2048-like: GPU pooled selection, then the GPU forward; 16 sampled rows of every head.
+
+    Each sampled row's block row of the GPU selection is first checked against the oracle's
+    pooled scores; only a row that passes becomes the oracle forward's mask."""
     m = bsa()
     w = W.c3()
     shp = w["shape"]
@@ -233,9 +266,11 @@ def test_forward_c3_sampled_rows_with_gpu_selection():
     assert m.get_device_error() == 0
     bm = blocks.bitmap.cpu().numpy()
     rng = np.random.default_rng(0)
-    for h in range(0, shp.H, 3):
-        rows = np.sort(rng.choice(shp.N, 64, replace=False))
+    for h in range(shp.H):
+        rows = np.unique(np.concatenate([[0, shp.N - 1], rng.choice(shp.N, 14, replace=False)]))
+        qh, kh = f64(w["q"][0, h]), f64(w["k"][0, h])
+        check_pooled_rows(bm[0, h], qh, kh, shp.block_q, shp.block_k, shp.n_text, w["groups"],
+                          np.unique(rows // shp.block_q))
         fn = OA.block_mask_to_token_fn(bm[0, h], 128, 128, shp.N)
-        exp = OA.head_forward(f64(w["q"][0, h]), f64(w["k"][0, h]), f64(w["v"][0, h]), 1, fn, 128 ** -0.5,
-                              rows=rows)
+        exp = OA.head_forward(qh, kh, f64(w["v"][0, h]), 1, fn, 128 ** -0.5, rows=rows)
         assert_close_out(f64(o[0, h])[rows], exp, f"c3 h{h}")

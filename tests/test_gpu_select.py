@@ -6,7 +6,7 @@ import torch
 import workloads as W
 from oracle import masks as OM
 from oracle import select as OS
-from parity_util import bsa, f64, list_to_classes, selection_matches
+from parity_util import bsa, check_full_score_rows, f64, list_to_classes, selection_matches
 
 pytestmark = pytest.mark.gpu
 
@@ -113,11 +113,38 @@ def test_full_score_select_zero_q_takes_lowest_indices():
         assert list(np.nonzero(cls[0, 0, I])[0]) == [0, 1, 4]
 
 
+def c4_rows_plan(kinds, n_qb, n_full_heads=4, rows_per_head=16, seed=0):
+    """Which query-block rows of each head the 32k check compares: every row of two 'column' and
+    two 'slide-window' heads (or the first heads if one kind is missing), and a seeded 16 rows of
+    every other head that always include the first row and the last one (a generation row)."""
+    col = [h for h, kd in enumerate(kinds) if kd[0] == "column"]
+    win = [h for h, kd in enumerate(kinds) if kd[0] != "column"]
+    full = (col[:n_full_heads // 2] + win[:n_full_heads // 2])
+    full += [h for h in range(len(kinds)) if h not in full][:n_full_heads - len(full)]
+    rng = np.random.default_rng(seed)
+    plan = {}
+    for h in range(len(kinds)):
+        if h in full:
+            plan[h] = np.arange(n_qb)
+        else:
+            extra = rng.choice(np.arange(1, n_qb - 1), rows_per_head - 2, replace=False)
+            plan[h] = np.unique(np.concatenate([[0, n_qb - 1], extra]))
+    return plan
+
+
 @pytest.mark.slow
-def test_full_score_select_c4_sampled_rows():
+def test_full_score_select_c4_rows():
+    """SparseD-like 32k selection: every query-block row of four heads (both bias kinds) and 16
+    rows of each of the other 28 heads against the oracle's A' (isolated prefill / generation
+    top-rho%, ties within 1e-5 relative excluded)."""
     w = W.c4()
     shp = w["shape"]
     q, k, _ = W.dlm_step_qkv(shp, 3, 0)
     cls = _select(shp, q, k, bsa().SELECT_FULL_SCORE, w["groups"], False, shp.d ** -0.5, w["bias"])
     assert (cls[0] > 0).sum(axis=-1).min() == 77 and (cls[0] > 0).sum(axis=-1).max() == 77
-    _check_full(shp, q, k, w["groups"], w["bias"], cls, rows_per_head=2)
+    plan = c4_rows_plan(w["bias_kinds"], shp.n_qb)
+    assert sum(len(r) == shp.n_qb for r in plan.values()) == 4
+    assert all(len(r) >= 16 for r in plan.values())
+    for h, rows in plan.items():
+        check_full_score_rows(cls[0, h], f64(q[0, h]), f64(k[0, h]), shp.d ** -0.5, shp.block_q, shp.block_k,
+                              w["groups"], rows, bias=w["bias"][h].numpy())

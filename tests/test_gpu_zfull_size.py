@@ -10,7 +10,7 @@ import torch
 
 import workloads as W
 from oracle import attention as OA
-from parity_util import assert_close_out, bsa, f64
+from parity_util import assert_close_out, bsa, check_full_score_rows, f64
 from test_gpu_forward import _check_arrow, _dims, _run_arrow
 
 pytestmark = pytest.mark.gpu
@@ -19,7 +19,8 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.slow
 def test_forward_c4_sampled_rows_with_gpu_selection():
     """SparseD-like DLM at 32k: the GPU full-score selection on step 0's Q/K, then the GPU forward
-    of step 1 reusing it with the block bias (the bench's launch); oracle on sampled rows."""
+    of step 1 reusing it with the block bias (the bench's launch); oracle on 16 sampled rows of
+    every head, each of whose selection rows is first checked against the oracle's A'."""
     m = bsa()
     w = W.c4()
     shp = w["shape"]
@@ -40,8 +41,11 @@ def test_forward_c4_sampled_rows_with_gpu_selection():
     bm = blocks.bitmap.cpu().numpy()
     bias_np = bias.numpy()
     rng = np.random.default_rng(1)
-    for h in range(0, shp.H, 4):
-        rows = np.sort(rng.choice(shp.N, 32, replace=False))
+    for h in range(shp.H):
+        rows = np.unique(np.concatenate([[0, shp.N - 1], rng.choice(shp.N, 14, replace=False)]))
+        # the GPU selection rows these query rows use must first agree with the oracle's A' of step 0
+        check_full_score_rows(bm[0, h], f64(q0[0, h]), f64(k0[0, h]), shp.d ** -0.5, shp.block_q, shp.block_k,
+                              w["groups"], np.unique(rows // shp.block_q), bias=bias_np[h])
         fn = OA.block_mask_to_token_fn(bm[0, h], 128, 128, shp.N)
         bfn = OA.block_bias_fn(bias_np[h], 128, 128, shp.N)
         exp = OA.head_forward(f64(q1[0, h]), f64(k1[0, h]), f64(v1[0, h]), 1, fn, 128 ** -0.5, rows=rows,

@@ -40,6 +40,10 @@ extern "C" int h_gna_classes(int n_text, const bsa_gna_geom* geom, unsigned char
     for (int J = 0; J < nb; ++J) out[I * nb + J] = (unsigned char)bsa::gna_class(g, I, J);
   return 0;
 }
+extern "C" void h_fdiv_many(int d, const int* n, long long* out, int count) {
+  const bsa::FastDiv f = bsa::make_fastdiv(d);
+  for (int i = 0; i < count; ++i) out[i] = bsa::fdiv(n[i], f);
+}
 extern "C" int h_tile_sources(int n_text, const bsa_gna_geom* geom, int* out, int n) {
   bsa::GnaDev g;
   const int st = bsa::make_gna(geom, n_text, &g);
@@ -67,7 +71,25 @@ def host_lib(tmp_path_factory):
     lib.h_segbits_row.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
     lib.h_tile_sources.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.h_gna_classes.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    lib.h_fdiv_many.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return lib
+
+
+def test_division_by_invariant_integers_is_exact(host_lib):
+    """The fine mask divides by launch invariants with a multiply-high and a shift (Granlund and
+    Montgomery, N = 31): exact floor division for every divisor up to 4096 over all dividends
+    below 2^20, and for large dividends up to 2^31 - 1 (also with large divisors)."""
+    rng = np.random.default_rng(0)
+    dense = np.arange(0, 1 << 20, dtype=np.int32)
+    big = np.concatenate([rng.integers(0, 2 ** 31 - 1, 20000),
+                          np.arange(2 ** 31 - 2048, 2 ** 31, dtype=np.int64)]).astype(np.int32)
+    out = np.empty(len(dense), dtype=np.int64)
+    divisors = list(range(1, 4097)) + [65535, 65536, 100003, 1 << 20, (1 << 30) + 7, 2 ** 31 - 1]
+    for d in divisors:
+        for n in ((dense, big) if d <= 256 else (dense[::61], big)):
+            n = np.ascontiguousarray(n)
+            host_lib.h_fdiv_many(d, n.ctypes.data, out.ctypes.data, len(n))
+            assert np.array_equal(out[:len(n)], n.astype(np.int64) // d), d
 
 
 class Geom(ctypes.Structure):  # bsa_gna_geom
