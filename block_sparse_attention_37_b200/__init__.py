@@ -29,6 +29,7 @@ EXPORTS = (
     "bsa_select_topk", "bsa_forward", "bsa_gna_tiled_len", "bsa_permute_tiles",
     "bsa_unpermute_tiles", "bsa_get_device_error", "bsa_select_topk_static", "bsa_rse",
     "bsa_plan_heads", "bsa_schedule_full_steps", "bsa_step_action", "bsa_keep_pct", "bsa_jaccard",
+    "bsa_set_wait_limit_ns", "bsa_set_withheld_tile",
 )
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -114,6 +115,8 @@ def _lib():
         lib.bsa_step_action.argtypes = [I32, I32, I32, P]
         lib.bsa_keep_pct.argtypes = [I32, I32, I32, I32, I32, I32, P]
         lib.bsa_jaccard.argtypes = [P, P, P, P, P]
+        lib.bsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.bsa_set_withheld_tile.argtypes = [I32]
         _LIB = lib
     return _LIB
 
@@ -402,6 +405,16 @@ def jaccard(dm: Dims, a: BlockList, b: BlockList, out, stream=None):
     ca, cb = a.c(dm, p[0:4]), b.c(dm, p[4:8])
     _check(_lib().bsa_jaccard(ctypes.byref(dm), ctypes.byref(ca), ctypes.byref(cb), p[8], _stream(stream)),
            "bsa_jaccard")
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    """Bound of every pipeline wait in later forward / full-score selection launches (0: default 2 s)."""
+    _check(_lib().bsa_set_wait_limit_ns(int(ns)), "bsa_set_wait_limit_ns")
+
+
+def set_withheld_tile(tile: int) -> None:
+    """Test hook: later forwards never load this key tile's K, so its waits run out (-1: off)."""
+    _check(_lib().bsa_set_withheld_tile(int(tile)), "bsa_set_withheld_tile")
 
 
 def get_device_error(stream=None) -> int:

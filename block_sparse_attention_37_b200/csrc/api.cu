@@ -1,6 +1,7 @@
 // C ABI of the library (include/bsa.h): argument checks, TMA descriptors and
 // launches. No allocation, no host synchronisation except in
 // bsa_get_device_error, no CPU fallback.
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -17,6 +18,11 @@ namespace {
 constexpr int kVersion = 100;  // 0.1.0
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+// Failure-detection settings read by every later launch (bsa_set_wait_limit_ns,
+// bsa_set_withheld_tile).
+std::atomic<uint64_t> g_wait_limit_ns{kWaitLimitNs};
+std::atomic<int> g_withheld_tile{-1};
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -303,6 +309,8 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K, const bs
     ap.nSeg = ceil_div(dims->N, 64);
     ap.bias = block_bias;
     ap.scale_log2 = spec->scale * 1.4426950408889634f;
+    ap.wait_limit_ns = g_wait_limit_ns.load();
+    ap.withhold_tile = -1;
     ap.lse = reinterpret_cast<float*>(ws + L.lse);
     ap.apool = reinterpret_cast<float*>(ws + L.apool);
     const int grid = (int)(BH * ap.nQT);
@@ -367,6 +375,8 @@ int bsa_forward(const bsa_dims* dims, const void* Q, const void* K, const void* 
   ap.bias = block_bias;
   ap.scale_log2 = scale * 1.4426950408889634f;
   ap.O = static_cast<__nv_bfloat16*>(O);
+  ap.wait_limit_ns = g_wait_limit_ns.load();
+  ap.withhold_tile = g_withheld_tile.load();
   const long long grid = BH * ceil_div(dims->N, 256);
   if (grid > 0x7fffffffll) return BSA_ERR_UNSUPPORTED;
   return cuda_status(launch_forward(dims->d, mq, mk, mv, mo, ap, (int)grid, static_cast<cudaStream_t>(stream)));
@@ -405,6 +415,17 @@ int bsa_permute_tiles(const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_
 int bsa_unpermute_tiles(const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_tensors, const void* const* in,
                         void* const* out, void* stream) {
   return permute_common(false, dims, geom, n_tensors, in, out, stream);
+}
+
+int bsa_set_wait_limit_ns(uint64_t ns) {
+  g_wait_limit_ns.store(ns == 0 ? kWaitLimitNs : ns);
+  return BSA_OK;
+}
+
+int bsa_set_withheld_tile(int32_t tile) {
+  if (tile < -1) return BSA_ERR_INVALID_ARG;
+  g_withheld_tile.store(tile);
+  return BSA_OK;
 }
 
 int bsa_get_device_error(void* stream, int32_t* code) {

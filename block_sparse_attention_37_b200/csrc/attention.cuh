@@ -29,6 +29,10 @@ struct AttnParams {
   float* apool;              // [B,H,nQB,nKB] block sums of softmax (POOL out)
   int has_gna;
   GnaDev g;
+  // failure detection: the limit of every pipeline wait, and a tile whose K
+  // the producer withholds (-1: none) so that a test can make a wait run out
+  uint64_t wait_limit_ns;
+  int withhold_tile;
 };
 
 // The forward: two 128-row query tiles per CTA (forward.cu); grid = B*H*ceil(N/256).

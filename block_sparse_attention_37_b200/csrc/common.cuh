@@ -108,13 +108,17 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Upper bound on any single pipeline wait. A correct kernel waits microseconds;
-// after this long the wait gives up, the CTA aborts and the error word is set.
+// Default upper bound on any single pipeline wait. A correct kernel waits
+// microseconds; after this long the wait gives up, the CTA aborts and the
+// error word is set. The caller may shorten it (bsa_set_wait_limit_ns); the
+// drains of an aborting CTA (copies and MMAs already in flight, which always
+// complete) keep this bound.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 // Wait until the phase of `bar` with parity `parity` has completed. Returns
-// false when the CTA's abort flag is raised or the time limit runs out.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// false when the CTA's abort flag is raised or `limit_ns` runs out.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -122,8 +126,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+  }
+}
+
+// Drain wait of an aborting CTA: until the phase completes or the default
+// bound runs out (the abort flag is not consulted).
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(a, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {
   }
 }
 

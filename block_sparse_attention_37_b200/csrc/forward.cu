@@ -39,7 +39,7 @@ struct FwdCfg {
   static constexpr int K_OFF = 2 * TILE;
   static constexpr int V_OFF = K_OFF + STAGES * TILE;
   static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
-  static constexpr int NBAR = 2 + 6 * STAGES + 8;
+  static constexpr int NBAR = 2 + 6 * STAGES + 8 + 1;
   // d = 64: P gets its own tensor-memory columns (S 128 + P 64 + O 64 per
   // warpgroup fill all 512), so the next QK^T can overwrite S as soon as the
   // softmax has read it; d = 128: P is written over S and waits for PV.
@@ -382,6 +382,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* p_full = s_full + 2;    // [2]
   uint64_t* o_ready = p_full + 2;   // [2]
   uint64_t* s_free = o_ready + 2;   // [2] (separate-P layout: S read by the softmax)
+  uint64_t* mma_done = s_free + 2;  // every MMA of the CTA complete (teardown)
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   uint32_t* vb = reinterpret_cast<uint32_t*>(smem + C::BITS_OFF);
@@ -395,6 +396,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&o_ready[w], 1);
       mbar_init(&s_free[w], 128);
     }
+    mbar_init(mma_done, 1);
     for (int s = 0; s < S; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
@@ -482,24 +484,28 @@ __global__ void __launch_bounds__(384, 1)
         for (int w = 0; w < 2 && released; ++w)
           if ((prev_need >> w) & 1) {
             const int b = 2 * st + w;
-            released = mbar_wait(&k_empty[b], (kpar >> b) & 1u, abort_flag);
+            released = mbar_wait(&k_empty[b], (kpar >> b) & 1u, abort_flag, p.wait_limit_ns);
             kpar ^= 1u << b;
           }
         if (!released) {
           cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
           break;
         }
-        mbar_arrive_expect_tx(&k_full[st], C::TILE);
-        uint8_t* dk = sK + st * C::TILE;
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(dk + c * C::CHUNK, &tmK, &k_full[st], c * 64, sa * 64, bh);
-          tma_load_3d(dk + c * C::CHUNK + C::CHUNK / 2, &tmK, &k_full[st], c * 64, sb * 64, bh);
+        // a withheld tile (failure-detection test) is never loaded: its
+        // consumers' waits run out
+        if (t != p.withhold_tile) {
+          mbar_arrive_expect_tx(&k_full[st], C::TILE);
+          uint8_t* dk = sK + st * C::TILE;
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(dk + c * C::CHUNK, &tmK, &k_full[st], c * 64, sa * 64, bh);
+            tma_load_3d(dk + c * C::CHUNK + C::CHUNK / 2, &tmK, &k_full[st], c * 64, sb * 64, bh);
+          }
         }
         k_issued = t + 1;
         for (int w = 0; w < 2 && released; ++w)
           if ((prev_need >> w) & 1) {
             const int b = 2 * st + w;
-            released = mbar_wait(&v_empty[b], (vpar >> b) & 1u, abort_flag);
+            released = mbar_wait(&v_empty[b], (vpar >> b) & 1u, abort_flag, p.wait_limit_ns);
             vpar ^= 1u << b;
           }
         if (!released) {
@@ -514,24 +520,15 @@ __global__ void __launch_bounds__(384, 1)
         }
         v_issued = t + 1;
       }
-      if (*abort_flag) {
-        const uint64_t t0 = globaltimer_ns();
-        auto drain = [&](uint64_t* bar, uint32_t ph) {
-          while (!mbar_try_wait(smem_u32(bar), ph) && globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
-        };
+      if (*abort_flag) {  // copies in flight land before the CTA ends
         for (int t = k_issued - S < 0 ? 0 : k_issued - S; t < k_issued; ++t)
-          drain(&k_full[t % S], (uint32_t)(t / S) & 1u);
+          if (t != p.withhold_tile) mbar_drain(&k_full[t % S], (uint32_t)(t / S) & 1u);
         for (int t = v_issued - S < 0 ? 0 : v_issued - S; t < v_issued; ++t)
-          drain(&v_full[t % S], (uint32_t)(t / S) & 1u);
+          mbar_drain(&v_full[t % S], (uint32_t)(t / S) & 1u);
       }
     }
-    if (lane == 0) {  // every CTA loaded Q: it must have landed before the CTA ends
-      const uint64_t t0 = globaltimer_ns();
-      for (int w = 0; w < 2; ++w)
-        while (!mbar_try_wait(smem_u32(&q_full[w]), 0u) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
-    }
+    if (lane == 0)  // every CTA loaded Q: it must have landed before the CTA ends
+      for (int w = 0; w < 2; ++w) mbar_drain(&q_full[w], 0u);
     } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     // Two issue strategies, chosen by what measured faster for each layout.
@@ -634,11 +631,17 @@ __global__ void __launch_bounds__(384, 1)
           if ((++spins & 63u) == 0) {
             const uint64_t now = __shfl_sync(0xffffffffu, globaltimer_ns(), 0);
             if (spins == 64) t_idle = now;
-            if (__any_sync(0xffffffffu, *abort_flag != 0) || now - t_idle > kWaitLimitNs) {
+            if (__any_sync(0xffffffffu, *abort_flag != 0) || now - t_idle > p.wait_limit_ns) {
               cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
               break;
             }
           }
+        }
+        // tensor memory is freed only once every issued MMA has completed (an
+        // aborting CTA may leave MMAs in flight)
+        if (g0.cnt + g1.cnt > 0) {
+          tc_commit_warp(mma_done);
+          mbar_drain(mma_done, 0u);
         }
       }
     } else {
@@ -653,7 +656,7 @@ __global__ void __launch_bounds__(384, 1)
         constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
         const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
-          return warp_all(mbar_wait(bar, parity, abort_flag));
+          return warp_all(mbar_wait(bar, parity, abort_flag, p.wait_limit_ns));
         };
         // per warpgroup: tile whose PV is outstanding (-1: none) and its index
         // among the warpgroup's tiles; QK^T issued so far
@@ -722,6 +725,12 @@ __global__ void __launch_bounds__(384, 1)
         }
         ok = ok && flush_below(T);
         if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+        // tensor memory is freed only once every issued MMA has completed (an
+        // aborting CTA may leave MMAs in flight)
+        if (c0 + c1 > 0) {
+          tc_commit_warp(mma_done);
+          mbar_drain(mma_done, 0u);
+        }
       }
     }
     }
@@ -751,7 +760,7 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       if (!((tile_need(sched, nseg, t, act) >> w) & 1)) continue;
-      ok = warp_all(mbar_wait(&s_full[w], (uint32_t)j & 1u, abort_flag));
+      ok = warp_all(mbar_wait(&s_full[w], (uint32_t)j & 1u, abort_flag, p.wait_limit_ns));
       if (!ok) break;
       tc_fence_after();
       const int ea = sched[2 * t];
@@ -836,7 +845,7 @@ __global__ void __launch_bounds__(384, 1)
       // over S at d = 128) and before O is rescaled; O is rescaled once S is
       // dead (fewer live registers), which is safe because PV(j) waits for p_full
       if (j > 0) {
-        ok = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
+        ok = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag, p.wait_limit_ns));
         if (!ok) break;
         tc_fence_after();
       }
@@ -863,10 +872,11 @@ __global__ void __launch_bounds__(384, 1)
     // ---------------------------------------------------------------- epilogue
     // O is staged over the Q tile: a warpgroup that computed nothing has not
     // seen Q land yet
-    if (j == 0 && !warp_all(mbar_wait(&q_full[w], 0u, abort_flag))) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+    if (j == 0 && !warp_all(mbar_wait(&q_full[w], 0u, abort_flag, p.wait_limit_ns)))
+      cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
     bool have = ok && j > 0;
     if (have) {
-      have = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag));
+      have = warp_all(mbar_wait(&o_ready[w], (uint32_t)(j - 1) & 1u, abort_flag, p.wait_limit_ns));
       if (!have) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
       tc_fence_after();
     }

@@ -24,7 +24,8 @@ struct ScoreCfg {
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = TILE_BYTES;
   static constexpr int BAR_OFF = K_OFF + STAGES * TILE_BYTES;
-  static constexpr int NBAR = 1 + 2 * STAGES + 4;  // q_full, k_full[S], k_empty[S], s_full[2], s_free[2]
+  // q_full, k_full[S], k_empty[S], s_full[2], s_free[2], mma_done
+  static constexpr int NBAR = 1 + 2 * STAGES + 4 + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* k_empty = k_full + S;
   uint64_t* s_full = k_empty + S;
   uint64_t* s_free = s_full + 2;
+  uint64_t* mma_done = s_free + 2;  // every MMA of the CTA complete (teardown)
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
 
@@ -68,6 +70,7 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&s_full[b], 1);
       mbar_init(&s_free[b], 128);
     }
+    mbar_init(mma_done, 1);
     misc[1] = 0;
     fence_barrier_init();
   }
@@ -91,7 +94,7 @@ __global__ void __launch_bounds__(192, 1)
       int issued = 0;
       for (int t = 0; t < T; ++t) {
         const int st = t % S;
-        if (t >= S && !mbar_wait(&k_empty[st], ((uint32_t)(t / S) & 1u) ^ 1u, abort_flag)) {
+        if (t >= S && !mbar_wait(&k_empty[st], ((uint32_t)(t / S) & 1u) ^ 1u, abort_flag, p.wait_limit_ns)) {
           cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
           break;
         }
@@ -103,25 +106,21 @@ __global__ void __launch_bounds__(192, 1)
                         t * 128 + 64 * r, bh);
         issued = t + 1;
       }
-      if (*abort_flag) {
-        const uint64_t t0 = globaltimer_ns();
-        while (!mbar_try_wait(smem_u32(q_full), 0u) && globaltimer_ns() - t0 < kWaitLimitNs) {
-        }
-        for (int t = issued - S < 0 ? 0 : issued - S; t < issued; ++t)
-          while (!mbar_try_wait(smem_u32(&k_full[t % S]), (uint32_t)(t / S) & 1u) &&
-                 globaltimer_ns() - t0 < kWaitLimitNs) {
-          }
+      if (*abort_flag) {  // copies in flight land before the CTA ends
+        mbar_drain(q_full, 0u);
+        for (int t = issued - S < 0 ? 0 : issued - S; t < issued; ++t) mbar_drain(&k_full[t % S], (uint32_t)(t / S) & 1u);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK);
-      bool ok = mbar_wait(q_full, 0u, abort_flag);
+      bool ok = mbar_wait(q_full, 0u, abort_flag, p.wait_limit_ns);
+      int issued = 0;
       for (int t = 0; t < T && ok; ++t) {
         const int st = t % S, buf = t & 1;
-        if (t >= 2) ok = mbar_wait(&s_free[buf], (uint32_t)((t - 2) >> 1) & 1u, abort_flag);
-        ok = ok && mbar_wait(&k_full[st], (uint32_t)(t / S) & 1u, abort_flag);
+        if (t >= 2) ok = mbar_wait(&s_free[buf], (uint32_t)((t - 2) >> 1) & 1u, abort_flag, p.wait_limit_ns);
+        ok = ok && mbar_wait(&k_full[st], (uint32_t)(t / S) & 1u, abort_flag, p.wait_limit_ns);
         if (!ok) break;
         tc_fence_after();
         const uint32_t kbase = sKa + st * C::TILE_BYTES;
@@ -133,8 +132,15 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_commit(&s_full[buf]);
         tc_commit(&k_empty[st]);
+        issued = t + 1;
       }
       if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
+      // tensor memory is freed only once every issued MMA has completed (an
+      // aborting CTA may leave MMAs in flight)
+      if (issued > 0) {
+        tc_commit(mma_done);
+        mbar_drain(mma_done, 0u);
+      }
     }
   } else {
     const int q4 = warp & 3;
@@ -150,7 +156,7 @@ __global__ void __launch_bounds__(192, 1)
     float s[128];
     for (int t = 0; t < T; ++t) {
       const int buf = t & 1;
-      ok = warp_all(mbar_wait(&s_full[buf], (uint32_t)(t >> 1) & 1u, abort_flag));
+      ok = warp_all(mbar_wait(&s_full[buf], (uint32_t)(t >> 1) & 1u, abort_flag, p.wait_limit_ns));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll

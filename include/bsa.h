@@ -308,6 +308,25 @@ int bsa_jaccard(const bsa_dims* dims, const bsa_block_list* a, const bsa_block_l
  * synchronisation itself failed. */
 int bsa_get_device_error(void* stream, int32_t* code);
 
+/* Failure detection (the pages have none; this is the library's own). Every
+ * pipeline wait inside bsa_forward and bsa_select_topk's full-score passes is
+ * bounded: a wait that runs out raises BSA_DEVERR_TIMEOUT in the device error
+ * word and its CTA aborts: copies and tensor-core operations already in
+ * flight are drained (under the default bound), tensor memory is freed and
+ * the CTA exits, so the context stays usable. Both settings below are
+ * process-wide and apply to calls made after them.
+ *
+ * bsa_set_wait_limit_ns: the bound of each pipeline wait, in nanoseconds;
+ * 0 restores the default of 2 s. Always returns BSA_OK. */
+int bsa_set_wait_limit_ns(uint64_t ns);
+
+/* bsa_set_withheld_tile: for tests of the above. When tile >= 0, every
+ * bsa_forward CTA that has a key tile with that index in its schedule never
+ * loads that tile's K, so the waits on it run out (after the wait limit) and
+ * the forward ends with BSA_DEVERR_TIMEOUT and an undefined O. -1 (the
+ * default) turns it off. Errors: INVALID_ARG for tile < -1. */
+int bsa_set_withheld_tile(int32_t tile);
+
 #ifdef __cplusplus
 }
 #endif

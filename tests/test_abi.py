@@ -109,6 +109,10 @@ def test_host_argument_checks_return_before_launch():
     assert lib.bsa_jaccard(ctypes.byref(dm), ctypes.byref(lst2), ctypes.byref(lst2), None, None) \
         == bsa.ERR_INVALID_ARG
     assert lib.bsa_error_string(bsa.ERR_INFEASIBLE) == b"no plan meets the error budget"
+    # failure-detection settings: host-only, no launch
+    assert lib.bsa_set_withheld_tile(-2) == bsa.ERR_INVALID_ARG
+    assert lib.bsa_set_withheld_tile(-1) == bsa.OK
+    assert lib.bsa_set_wait_limit_ns(0) == bsa.OK
 
 
 @pytest.mark.parametrize("n_text,grid,tile", [(256, (16, 48, 80), (4, 8, 8)), (5, (3, 5, 6), (2, 2, 4)),
