@@ -54,6 +54,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
+    ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: independent replicas per GPU (weak scaling, default), or one problem split "
+                         "by heads with O all-gathered inside every step (strong scaling)")
     a = ap.parse_args()
     steps, warmup = DEFAULT_STEPS[a.config]
     a.steps = steps if a.steps is None else a.steps
@@ -432,6 +435,15 @@ def rank_seed(cfg: str, rank: int) -> int:
     return DEFAULT_SEEDS[cfg] + 1000 * rank
 
 
+def reduce_sum(vals, world: int, device) -> list:
+    """Element-wise sum over ranks (the units of a head-sharded problem)."""
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
+
+
 def reduce_max(vals, world: int, device) -> list:
     """Element-wise max over ranks (timing only; the data path has no collective)."""
     t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
@@ -439,6 +451,56 @@ def reduce_max(vals, world: int, device) -> list:
         import torch.distributed as dist
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return [float(x) for x in t.tolist()]
+
+
+def shard_workload(w, rank: int, world: int):
+    """The rank's share of one problem split by heads: every per-head input sliced to the rank's
+    contiguous head range (block_sparse_attention_37_b200.sharding)."""
+    from block_sparse_attention_37_b200 import sharding
+    h0, h1 = sharding.head_range(w["shape"].H, rank, world)
+    out = dict(w)
+    for key in ("q", "k", "v", "cache"):
+        if out.get(key) is not None:
+            out[key] = sharding.local_heads(out[key], rank, world)
+    for key in ("head_mode", "window"):
+        if key in out:
+            out[key] = np.ascontiguousarray(out[key][h0:h1])
+    if "bias" in out:
+        out["bias"] = sharding.local_heads(out["bias"], rank, world, head_dim=0)
+    if "bias_kinds" in out:
+        out["bias_kinds"] = out["bias_kinds"][h0:h1]
+    out["shape"] = W.Shape(**{**out["shape"].__dict__, "H": h1 - h0})
+    return out
+
+
+class HeadShardedJob(Job):
+    """One rank's share of a problem split by heads: its heads' whole hot path, then the
+    all-gather of O (one NCCL all-gather per batch item) so every rank ends with every head."""
+
+    def __init__(self, job, world):
+        self.job, self.world = job, world
+        self.s = job.s
+        self.launches_per_step = job.launches_per_step
+        o = job.e2e_output()
+        self.full = torch.empty((o.shape[0], o.shape[1] * world) + tuple(o.shape[2:]), dtype=o.dtype,
+                                device=o.device)
+
+    def step(self, ev_fwd=None):
+        from block_sparse_attention_37_b200 import sharding
+        self.job.step(ev_fwd)
+        sharding.gather_heads(self.job.e2e_output(), self.world, out=self.full)
+
+    def e2e_inputs(self):
+        return self.job.e2e_inputs()
+
+    def e2e_output(self):
+        return self.full
+
+    def e2e_step(self):
+        for dst, src in zip(self.e2e_inputs(), self.pin):
+            dst.copy_(src, non_blocking=True)
+        self.step()
+        self.o_host.copy_(self.full, non_blocking=True)
 
 
 def job_throughput(flops_per_step: float, world: int, ms_per_step: float) -> float:
@@ -717,9 +779,15 @@ def run_bsa(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     cfg = args.config
     desc, make, JobT = CONFIGS[cfg]
-    seed = rank_seed(cfg, rank)
+    sharded = args.shard == "heads" and world > 1
+    seed = DEFAULT_SEEDS[cfg] if sharded else rank_seed(cfg, rank)
     w = make(seed)
-    job = JobT(w)
+    if sharded:
+        w = shard_workload(w, rank, world)
+        job = HeadShardedJob(JobT(w), world)
+    else:
+        job = JobT(w)
+    inner = job.job if sharded else job
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
 
     sampler = ClockSampler(local_rank)
@@ -737,27 +805,32 @@ def run_bsa(args, rank, world, local_rank):
     total_ms, fwd_total = reduce_max([np.sum(step_ms), np.sum(fwd_ms)], world, "cuda")
     ms_per_step = total_ms / args.steps
     fwd_ms_mean = fwd_total / args.steps
-    value = job_throughput(job.flops, world, ms_per_step)
+    if sharded:  # one problem: the units are the sum of the ranks' shares, over the slowest rank
+        flops_all, computed_all, total_all = reduce_sum([inner.flops, inner.blocks_computed,
+                                                         inner.blocks_total], world, "cuda")
+        value = flops_all / (ms_per_step * 1e-3) / 1e12
+    else:
+        value = job_throughput(inner.flops, world, ms_per_step)
 
     extra = {}
     if not args.no_dense:
         dense = JobT(w, dense=True)
         d_step, d_fwd = time_steps(dense, max(10, args.steps // 4), args.warmup, flush)
-        sparsity = 1.0 - job.blocks_computed / job.blocks_total
+        sparsity = 1.0 - inner.blocks_computed / inner.blocks_total
         extra = {"dense_fwd_ms": float(np.mean(d_fwd)), "fwd_ms": fwd_ms_mean,
                  "speedup_vs_dense": float(np.mean(d_fwd)) / fwd_ms_mean,
                  "ideal_speedup": 1.0 / (1.0 - sparsity) if sparsity < 1 else None,
                  "block_sparsity": sparsity,
                  "dense_tflops": dense.flops / (float(np.mean(d_fwd)) * 1e-3) / 1e12}
         del dense
-    if isinstance(job, DlmJob):
-        extra["selection_ms"] = job.selection_ms
-    if hasattr(job, "useful_flops"):  # pairs the mask allows, partial tiles counted by their real pairs
-        extra["useful_tflops"] = job.useful_flops / (fwd_ms_mean * 1e-3) / 1e12
-        extra["useful_flops_per_step"] = job.useful_flops
-    if hasattr(job, "phases"):
+    if isinstance(inner, DlmJob):
+        extra["selection_ms"] = inner.selection_ms
+    if hasattr(inner, "useful_flops"):  # pairs the mask allows, partial tiles counted by their real pairs
+        extra["useful_tflops"] = inner.useful_flops / (fwd_ms_mean * 1e-3) / 1e12
+        extra["useful_flops_per_step"] = inner.useful_flops
+    if hasattr(inner, "phases"):
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
-        extra["hbm_phases"] = phase_bandwidth(job.phases(), flush, hbm)
+        extra["hbm_phases"] = phase_bandwidth(inner.phases(), flush, hbm)
         extra["hbm_peak_gbs"] = f"{hbm} ({peak_src} copy bandwidth)"
 
     e2e = None
@@ -774,7 +847,8 @@ def run_bsa(args, rank, world, local_rank):
         e1.record()
         torch.cuda.synchronize()
         (e2e_ms,) = reduce_max([e0.elapsed_time(e1) / n], world, "cuda")
-        e2e = {"value": job_throughput(job.flops, world, e2e_ms), "unit": UNIT,
+        e2e_value = flops_all / (e2e_ms * 1e-3) / 1e12 if sharded else job_throughput(inner.flops, world, e2e_ms)
+        e2e = {"value": e2e_value, "unit": UNIT,
                "h2d_bytes_per_step": int(job.h2d), "d2h_bytes_per_step": int(job.d2h),
                "ms_per_step": e2e_ms}
 
@@ -784,30 +858,34 @@ def run_bsa(args, rank, world, local_rank):
         cpu.pop("seconds", None)
 
     peak = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
-    achieved = job.flops / (fwd_ms_mean * 1e-3) / 1e12
+    achieved = inner.flops / (fwd_ms_mean * 1e-3) / 1e12
     key = f"attn_fwd_{cfg}"
     roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
             "frac": achieved / peak, "traffic": traffic_for(key),
             "kernel": f"bsa::fwd_kernel<{job.s.d}> (bsa_forward)",
             "peak_source": f"{peak_src} bf16 burst (kernel timed alone between L2 flushes)",
-            "algorithmic_flops_per_launch": job.flops}
+            "algorithmic_flops_per_launch": inner.flops}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded; shapes of the pages' workloads)",
         "config": {"workload": desc, "config": cfg,
                    "l2": "flushed before every step (256 MiB write), flush outside the timed events",
-                   "parallelism": f"independent replica per GPU x{world}", "seed": DEFAULT_SEEDS[cfg]},
+                   "parallelism": (f"one problem split by heads over {world} GPUs, O all-gathered (NCCL) "
+                                   "inside every step") if sharded else f"independent replica per GPU x{world}",
+                   "seed": DEFAULT_SEEDS[cfg]},
         "pct_of_bf16_peak": 100.0 * value / world / peak,
         "pct_of_bf16_sustained": 100.0 * value / world
         / peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]),
         "roofline": roof,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": job.launches_per_step * args.steps,
+        "gpu_launches": inner.launches_per_step * args.steps,
         "clocks": sampler.summary(),
         "wall_s_timed_region": wall1 - wall0,
-        "blocks_computed": job.blocks_computed, "blocks_total": job.blocks_total,
+        "blocks_computed": int(computed_all) if sharded else inner.blocks_computed,
+        "blocks_total": int(total_all) if sharded else inner.blocks_total,
     }
     line.update(extra)
     if rank == 0:

@@ -97,6 +97,11 @@ int make_gna(const bsa_gna_geom* in, int n_text, GnaDev* g) {
   g->f_tiles1 = make_fastdiv(g->tiles[1]);
   g->f_tile2 = make_fastdiv(g->tile[2]);
   g->f_tile1 = make_fastdiv(g->tile[1]);
+  const int tx = g->tile[2];
+  g->seg_one_slice = tx <= 64 && 64 % tx == 0 && g->tile[1] % (64 / tx) == 0;
+  g->x_rep = 0ull;
+  if (g->seg_one_slice)
+    for (int r = 0; r < 64 / tx; ++r) g->x_rep |= 1ull << (tx * r);
   g->has_padding = g->text_span > n_text;
   for (int d = 0; d < 3; ++d) g->has_padding |= (g->grid[d] % g->tile[d]) != 0;
   return BSA_OK;

@@ -356,6 +356,13 @@ struct GnaDev {
   // invariant divisors of the fine mask: tile volume, tiles along x, tiles along y,
   // tile x extent, tile y extent
   FastDiv f_vol, f_tiles2, f_tiles1, f_tile2, f_tile1;
+  // segments of 64 keys that lie inside one t-slice of a tile (the tile's x
+  // extent divides 64 and 64 / x-extent divides its y extent): their rows in
+  // the window are contiguous, so the fine mask is one x-mask replicated over
+  // the rows (x_rep = sum of 2^(x-extent * r) over the 64 / x-extent rows)
+  // and cut to the row range
+  int seg_one_slice;
+  uint64_t x_rep;
 };
 
 __host__ __device__ __forceinline__ int gna_window_start(int i, int L, int k, int s) {

@@ -100,7 +100,20 @@ __host__ __device__ __forceinline__ uint64_t gna_segment_bits(const GnaDev& g, i
   const int tlo = q.lo0, thi = q.hi0 < g.grid[0] ? q.hi0 : g.grid[0];
   const int ylo = q.lo1, yhi = q.hi1 < g.grid[1] ? q.hi1 : g.grid[1];
   uint64_t m = 0ull;
-  if (Tx <= 64) {
+  if (g.seg_one_slice) {
+    // one t-slice: t is fixed and the rows in the window form the range
+    // [rlo, rhi) of the segment's 64 / Tx rows
+    const int rows = 64 / Tx;
+    const int R0 = fdiv(l0, g.f_tile2);
+    const int tq = fdiv(R0, g.f_tile1);
+    const int t = bt + tq, y0 = by + (R0 - tq * Ty);
+    if (t >= tlo && t < thi) {
+      const int rlo = ylo - y0 > 0 ? ylo - y0 : 0;
+      const int rhi = yhi - y0 < rows ? yhi - y0 : rows;
+      const uint64_t xb = bit_range64(xlo - bx, xhi - bx) & bit_range64(0, Tx);
+      if (rlo < rhi) m = (xb * g.x_rep) & bit_range64(rlo * Tx, rhi * Tx);
+    }
+  } else if (Tx <= 64) {
     const int rows = 64 / Tx;  // Tx divides 64 (host check)
     const int R0 = fdiv(l0, g.f_tile2);
     int tq = fdiv(R0, g.f_tile1);

@@ -113,6 +113,8 @@ CASES = [
     (17, (6, 10, 12), (2, 2, 16), (4, 5, 6), (2, 1, 3)),        # mixed strides, ragged text
     (256, (16, 48, 80), (4, 8, 8), (8, 16, 24), (1, 1, 1)),     # the video workload, stride 1
     (256, (16, 48, 80), (4, 8, 8), (8, 16, 24), (4, 8, 8)),     # the video workload, stride 4x8x8
+    (33, (3, 37, 21), (1, 16, 8), (2, 9, 11), (1, 2, 3)),       # segments in one t-slice, two per slice
+    (0, (40, 50), (8, 8), (7, 9), (1, 1)),                      # 2-D, one segment per tile, padded y
 ]
 
 
