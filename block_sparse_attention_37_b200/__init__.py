@@ -29,7 +29,7 @@ EXPORTS = (
     "bsa_select_topk", "bsa_forward", "bsa_gna_tiled_len", "bsa_permute_tiles",
     "bsa_unpermute_tiles", "bsa_get_device_error", "bsa_select_topk_static", "bsa_rse",
     "bsa_plan_heads", "bsa_schedule_full_steps", "bsa_step_action", "bsa_keep_pct", "bsa_jaccard",
-    "bsa_set_wait_limit_ns", "bsa_set_withheld_tile",
+    "bsa_set_wait_limit_ns", "bsa_set_withheld_tile", "bsa_quantize_fp8", "bsa_forward_fp8",
 )
 STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -116,6 +116,8 @@ def _lib():
         lib.bsa_keep_pct.argtypes = [I32, I32, I32, I32, I32, I32, P]
         lib.bsa_jaccard.argtypes = [P, P, P, P, P]
         lib.bsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        lib.bsa_quantize_fp8.argtypes = [P] * 11
+        lib.bsa_forward_fp8.argtypes = [P] * 13 + [ctypes.c_float, P, P]
         lib.bsa_set_withheld_tile.argtypes = [I32]
         _LIB = lib
     return _LIB
@@ -306,6 +308,60 @@ def forward(dm: Dims, q, k, v, o, head_mode, blocks: BlockList | None = None, gn
     _check(_lib().bsa_forward(ctypes.byref(dm), qp, kp, vp, ctypes.byref(lc) if lc is not None else None, hm,
                               ctypes.byref(gna) if gna is not None else None, ci, co, bp, float(scale), op,
                               _stream(stream)), "bsa_forward")
+
+
+@dataclass
+class Fp8Operands:
+    """The e4m3 operands bsa_quantize_fp8 writes: codes of Q and K (uint8 [B, H, N, 128]), V's
+    codes transposed per head (uint8 [B, H, 128, Nt], Nt = N rounded up to 16) and the fp32
+    scales per 64-token block ([B, H, ceil(N / 64)])."""
+    q8: torch.Tensor
+    k8: torch.Tensor
+    v8t: torch.Tensor
+    sq: torch.Tensor
+    sk: torch.Tensor
+    sv: torch.Tensor
+
+    @staticmethod
+    def empty(B: int, H: int, N: int, d: int = 128, device="cuda") -> "Fp8Operands":
+        nt, ns = (N + 15) // 16 * 16, n_blocks(N, 64)
+        u8 = lambda *shape: torch.empty(shape, dtype=torch.uint8, device=device)
+        f32 = lambda: torch.empty((B, H, ns), dtype=torch.float32, device=device)
+        return Fp8Operands(u8(B, H, N, d), u8(B, H, N, d), u8(B, H, d, nt), f32(), f32(), f32())
+
+    def specs(self, dm: Dims):
+        n, nt, ns = _tokens(dm), (dm.N + 15) // 16 * 16, n_blocks(dm.N, 64)
+        bh = max(dm.B, 0) * max(dm.H, 0)
+        return [(self.q8, torch.uint8, "q8", n), (self.k8, torch.uint8, "k8", n),
+                (self.v8t, torch.uint8, "v8t", bh * dm.d * nt), (self.sq, torch.float32, "sq", bh * ns),
+                (self.sk, torch.float32, "sk", bh * ns), (self.sv, torch.float32, "sv", bh * ns)]
+
+
+def quantize_fp8(dm: Dims, q, k, v, ops: Fp8Operands, stream=None):
+    """bsa_quantize_fp8: e4m3 codes and per-64-token-block scales of q, k, v (cuda bf16
+    [B, H, N, 128]) into `ops` (Fp8Operands.empty(B, H, N))."""
+    n = _tokens(dm)
+    p = _ptrs((q, torch.bfloat16, "Q", n), (k, torch.bfloat16, "K", n), (v, torch.bfloat16, "V", n),
+              *ops.specs(dm))
+    _check(_lib().bsa_quantize_fp8(ctypes.byref(dm), *p, _stream(stream)), "bsa_quantize_fp8")
+
+
+def forward_fp8(dm: Dims, ops: Fp8Operands, o, head_mode, blocks: BlockList | None = None,
+                gna: GnaGeom | None = None, cache_in=None, cache_out=None, bias=None, scale: float | None = None,
+                stream=None):
+    """bsa_forward_fp8: bsa_forward on the e4m3 operands of quantize_fp8; o is cuda bf16 [B, H, N, 128]."""
+    scale = (1.0 / dm.d ** 0.5) if scale is None else scale
+    n, (_, nQB, nKB) = _tokens(dm), _grid(dm)
+    ls = blocks.specs(dm) if blocks is not None else []
+    p = _ptrs(*ls, *ops.specs(dm), (o, torch.bfloat16, "O", n), (head_mode, torch.int32, "head_mode", dm.H),
+              (cache_in, torch.float32, "cache_in", n), (cache_out, torch.float32, "cache_out", n),
+              (bias, torch.float32, "bias", dm.H * nQB * nKB))
+    lc = blocks.c(dm, p[:4]) if blocks is not None else None
+    q8, k8, v8t, sq, sk, sv, op, hm, ci, co, bp = p[len(ls):]
+    _check(_lib().bsa_forward_fp8(ctypes.byref(dm), q8, k8, v8t, sq, sk, sv,
+                                  ctypes.byref(lc) if lc is not None else None, hm,
+                                  ctypes.byref(gna) if gna is not None else None, ci, co, bp, float(scale), op,
+                                  _stream(stream)), "bsa_forward_fp8")
 
 
 def gna_tiled_len(n_text: int, gna: GnaGeom) -> int:

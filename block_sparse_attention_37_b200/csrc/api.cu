@@ -8,6 +8,7 @@
 #include "attention.cuh"
 #include "mask.cuh"
 #include "permute.cuh"
+#include "quant.cuh"
 #include "select.cuh"
 
 namespace bsa {
@@ -61,6 +62,23 @@ int make_map(CUtensorMap* m, const void* base, long long BH, int N, int d) {
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? BSA_OK : BSA_ERR_CUDA;
 }
+
+// [BH, rows, inner] bytes (e4m3 codes) as a 3-D tensor; 128-byte x 64-row
+// boxes, 128-byte swizzle; reads past `rows` or `inner` give zero.
+int make_map8(CUtensorMap* m, const void* base, long long BH, int rows, int inner) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return BSA_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)rows, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)inner, (cuuint64_t)rows * inner};
+  cuuint32_t box[3] = {128, 64, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? BSA_OK : BSA_ERR_CUDA;
+}
+
+int round16(int n) { return (n + 15) & ~15; }
 
 int num_sms() {
   int dev = 0, n = 148;
@@ -170,6 +188,56 @@ int check_select_args(const bsa_dims* dims, const void* Q, const void* K, const 
     if (dims->block_q != dims->block_k || dims->block_q % 128 != 0) return BSA_ERR_UNSUPPORTED;
     if (ceil_div(dims->N, 64) > kMaxSeg) return BSA_ERR_UNSUPPORTED;
   }
+  return BSA_OK;
+}
+
+// The checks and parameters both forwards share (everything but the
+// operand maps). gna_vol_mult: the tile volume a GNA layout must be a
+// multiple of (64 for the bf16 forward, 128 for the e4m3 one).
+int forward_params(const bsa_dims* dims, const bsa_block_list* list, const int32_t* head_mode,
+                   const bsa_gna_geom* gna, const float* cache_in, float* cache_out, const float* block_bias,
+                   float scale, void* O, int gna_vol_mult, AttnParams* out) {
+  if (!O || !head_mode || !aligned16(O)) return BSA_ERR_INVALID_ARG;
+  if ((cache_in && !aligned16(cache_in)) || (cache_out && !aligned16(cache_out))) return BSA_ERR_INVALID_ARG;
+  if (ceil_div(dims->N, 64) > kMaxSeg) return BSA_ERR_UNSUPPORTED;
+  const int nQB = ceil_div(dims->N, dims->block_q), nKB = ceil_div(dims->N, dims->block_k);
+  if (list && (!list->cnt || !list->idx || !list->flag || list->max_k < 1)) return BSA_ERR_INVALID_ARG;
+  AttnParams& ap = *out;
+  std::memset(&ap, 0, sizeof(ap));
+  if (gna) {
+    int st = make_gna(gna, dims->n_text, &ap.g);
+    if (st != BSA_OK) return st;
+    if (tiled_len(ap.g) != dims->N || dims->block_q != ap.g.vol || dims->block_k != ap.g.vol)
+      return BSA_ERR_INVALID_ARG;
+    const int tx = ap.g.tile[2];
+    if (ap.g.vol % gna_vol_mult != 0 || !((tx <= 64 && 64 % tx == 0) || (tx > 64 && tx % 64 == 0)))
+      return BSA_ERR_UNSUPPORTED;
+    ap.has_gna = 1;
+  }
+  ap.B = dims->B;
+  ap.H = dims->H;
+  ap.N = dims->N;
+  ap.block_q = dims->block_q;
+  ap.block_k = dims->block_k;
+  ap.n_text = dims->n_text;
+  ap.nQB = nQB;
+  ap.nKB = nKB;
+  ap.nQT = ceil_div(dims->N, 128);
+  ap.nSeg = ceil_div(dims->N, 64);
+  if (list) {
+    ap.cnt = list->cnt;
+    ap.idx = list->idx;
+    ap.flag = list->flag;
+    ap.max_k = list->max_k;
+  }
+  ap.head_mode = head_mode;
+  ap.cache_in = cache_in;
+  ap.cache_out = cache_out;
+  ap.bias = block_bias;
+  ap.scale_log2 = scale * 1.4426950408889634f;
+  ap.O = static_cast<__nv_bfloat16*>(O);
+  ap.wait_limit_ns = g_wait_limit_ns.load();
+  ap.withhold_tile = g_withheld_tile.load();
   return BSA_OK;
 }
 
@@ -333,58 +401,78 @@ int bsa_forward(const bsa_dims* dims, const void* Q, const void* K, const void* 
                 const float* block_bias, float scale, void* O, void* stream) {
   int st = check_dims(dims);
   if (st != BSA_OK) return st;
-  if (!Q || !K || !V || !O || !head_mode) return BSA_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return BSA_ERR_INVALID_ARG;
-  if ((cache_in && !aligned16(cache_in)) || (cache_out && !aligned16(cache_out))) return BSA_ERR_INVALID_ARG;
+  if (!Q || !K || !V) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V)) return BSA_ERR_INVALID_ARG;
   if (dims->d != 64 && dims->d != 128) return BSA_ERR_UNSUPPORTED;
   if (dims->block_q % 64 != 0 || dims->block_k % 64 != 0) return BSA_ERR_UNSUPPORTED;
-  if (ceil_div(dims->N, 64) > kMaxSeg) return BSA_ERR_UNSUPPORTED;
-  const int nQB = ceil_div(dims->N, dims->block_q), nKB = ceil_div(dims->N, dims->block_k);
-  if (list && (!list->cnt || !list->idx || !list->flag || list->max_k < 1)) return BSA_ERR_INVALID_ARG;
   AttnParams ap;
-  std::memset(&ap, 0, sizeof(ap));
-  if (gna) {
-    if ((st = make_gna(gna, dims->n_text, &ap.g)) != BSA_OK) return st;
-    if (tiled_len(ap.g) != dims->N || dims->block_q != ap.g.vol || dims->block_k != ap.g.vol)
-      return BSA_ERR_INVALID_ARG;
-    const int tx = ap.g.tile[2];
-    if (ap.g.vol % 64 != 0 || !((tx <= 64 && 64 % tx == 0) || (tx > 64 && tx % 64 == 0)))
-      return BSA_ERR_UNSUPPORTED;
-    ap.has_gna = 1;
-  }
+  if ((st = forward_params(dims, list, head_mode, gna, cache_in, cache_out, block_bias, scale, O, 64, &ap)) != BSA_OK)
+    return st;
   const long long BH = (long long)dims->B * dims->H;
   CUtensorMap mq, mk, mv, mo;
   if ((st = make_map(&mq, Q, BH, dims->N, dims->d)) != BSA_OK) return st;
   if ((st = make_map(&mk, K, BH, dims->N, dims->d)) != BSA_OK) return st;
   if ((st = make_map(&mv, V, BH, dims->N, dims->d)) != BSA_OK) return st;
   if ((st = make_map(&mo, O, BH, dims->N, dims->d)) != BSA_OK) return st;
-  ap.B = dims->B;
-  ap.H = dims->H;
-  ap.N = dims->N;
-  ap.block_q = dims->block_q;
-  ap.block_k = dims->block_k;
-  ap.n_text = dims->n_text;
-  ap.nQB = nQB;
-  ap.nKB = nKB;
-  ap.nQT = ceil_div(dims->N, 128);
-  ap.nSeg = ceil_div(dims->N, 64);
-  if (list) {
-    ap.cnt = list->cnt;
-    ap.idx = list->idx;
-    ap.flag = list->flag;
-    ap.max_k = list->max_k;
-  }
-  ap.head_mode = head_mode;
-  ap.cache_in = cache_in;
-  ap.cache_out = cache_out;
-  ap.bias = block_bias;
-  ap.scale_log2 = scale * 1.4426950408889634f;
-  ap.O = static_cast<__nv_bfloat16*>(O);
-  ap.wait_limit_ns = g_wait_limit_ns.load();
-  ap.withhold_tile = g_withheld_tile.load();
   const long long grid = BH * ceil_div(dims->N, 256);
   if (grid > 0x7fffffffll) return BSA_ERR_UNSUPPORTED;
   return cuda_status(launch_forward(dims->d, mq, mk, mv, mo, ap, (int)grid, static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_quantize_fp8(const bsa_dims* dims, const void* Q, const void* K, const void* V, uint8_t* q8, uint8_t* k8,
+                     uint8_t* v8t, float* sq, float* sk, float* sv, void* stream) {
+  int st = check_dims(dims);
+  if (st != BSA_OK) return st;
+  const void* ptrs[6] = {Q, K, V, q8, k8, v8t};
+  for (const void* ptr : ptrs)
+    if (!ptr || !aligned16(ptr)) return BSA_ERR_INVALID_ARG;
+  if (!sq || !sk || !sv) return BSA_ERR_INVALID_ARG;
+  if (dims->d != 128) return BSA_ERR_UNSUPPORTED;
+  QuantParams p;
+  p.q = static_cast<const __nv_bfloat16*>(Q);
+  p.k = static_cast<const __nv_bfloat16*>(K);
+  p.v = static_cast<const __nv_bfloat16*>(V);
+  p.q8 = q8;
+  p.k8 = k8;
+  p.v8t = v8t;
+  p.sq = sq;
+  p.sk = sk;
+  p.sv = sv;
+  p.BH = (long long)dims->B * dims->H;
+  p.N = dims->N;
+  p.Nt = round16(dims->N);
+  p.nS = ceil_div(dims->N, 64);
+  if (p.BH > 65535) return BSA_ERR_UNSUPPORTED;  // grid y
+  return cuda_status(launch_quant_fp8(p, static_cast<cudaStream_t>(stream)));
+}
+
+int bsa_forward_fp8(const bsa_dims* dims, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t, const float* sq,
+                    const float* sk, const float* sv, const bsa_block_list* list, const int32_t* head_mode,
+                    const bsa_gna_geom* gna, const float* cache_in, float* cache_out, const float* block_bias,
+                    float scale, void* O, void* stream) {
+  int st = check_dims(dims);
+  if (st != BSA_OK) return st;
+  if (!q8 || !k8 || !v8t || !sq || !sk || !sv) return BSA_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return BSA_ERR_INVALID_ARG;
+  if (dims->d != 128) return BSA_ERR_UNSUPPORTED;
+  // every 128-key tile must be one aligned run of keys (the transposed V tile is one box)
+  if (dims->block_q % 64 != 0 || dims->block_k % 128 != 0) return BSA_ERR_UNSUPPORTED;
+  AttnParams ap;
+  if ((st = forward_params(dims, list, head_mode, gna, cache_in, cache_out, block_bias, scale, O, 128, &ap)) !=
+      BSA_OK)
+    return st;
+  ap.sq = sq;
+  ap.sk = sk;
+  ap.sv = sv;
+  const long long BH = (long long)dims->B * dims->H;
+  CUtensorMap mq, mk, mvt, mo;
+  if ((st = make_map8(&mq, q8, BH, dims->N, 128)) != BSA_OK) return st;
+  if ((st = make_map8(&mk, k8, BH, dims->N, 128)) != BSA_OK) return st;
+  if ((st = make_map8(&mvt, v8t, BH, 128, round16(dims->N))) != BSA_OK) return st;
+  if ((st = make_map(&mo, O, BH, dims->N, 128)) != BSA_OK) return st;
+  const long long grid = BH * ceil_div(dims->N, 256);
+  if (grid > 0x7fffffffll) return BSA_ERR_UNSUPPORTED;
+  return cuda_status(launch_forward_fp8(mq, mk, mvt, mo, ap, (int)grid, static_cast<cudaStream_t>(stream)));
 }
 
 static int permute_common(bool forward, const bsa_dims* dims, const bsa_gna_geom* geom, int32_t n_tensors,

@@ -33,11 +33,20 @@ struct AttnParams {
   // the producer withholds (-1: none) so that a test can make a wait run out
   uint64_t wait_limit_ns;
   int withhold_tile;
+  // e4m3 forward: dequantisation scales per 64-token block, [B*H, nSeg]
+  const float* sq;
+  const float* sk;
+  const float* sv;
 };
 
 // The forward: two 128-row query tiles per CTA (forward.cu); grid = B*H*ceil(N/256).
 cudaError_t launch_forward(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream);
+
+// The e4m3 forward (d = 128): Q and K codes [B*H, N, 128] bytes, V codes
+// transposed [B*H, 128, N rounded up to 16] bytes, scales in p.sq/sk/sv.
+cudaError_t launch_forward_fp8(const CUtensorMap& q8, const CUtensorMap& k8, const CUtensorMap& v8t,
+                               const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream);
 
 // The two score passes of the full-score selection (score.cu); grid = B*H*ceil(N/128).
 cudaError_t launch_score(int d, int kind, const CUtensorMap& q, const CUtensorMap& k, const AttnParams& p,

@@ -7,5 +7,6 @@
 #include "permute.cu"
 #include "select.cu"
 #include "select_static.cu"
+#include "quant.cu"
 #include "plan.cu"
 #include "schedule.cu"

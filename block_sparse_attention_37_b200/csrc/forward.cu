@@ -30,20 +30,26 @@ namespace bsa {
 
 constexpr float kRescaleTau = 8.0f;  // O is rescaled only when the row max grows by more than 2^8
 
-template <int D>
+// F8: the e4m3 form (d = 128 only). A 128-row tile of e4m3 codes is 128 rows
+// of 128 bytes, the byte geometry of a bf16 d = 64 tile, so four K/V stages
+// fit; the Q slots keep 32 KB each for the bf16 O staging; V arrives
+// transposed (K-major), one 128-byte run of keys per channel.
+template <int D, bool F8 = false>
 struct FwdCfg {
-  static constexpr int STAGES = D == 64 ? 4 : 2;
-  static constexpr int TILE = 128 * D * 2;
-  static constexpr int CHUNK = 128 * 128;  // 128 rows x 64 bf16
-  static constexpr int Q_OFF = 0;          // two Q tiles (reused as O staging)
-  static constexpr int K_OFF = 2 * TILE;
+  static constexpr int STAGES = (D == 64 || F8) ? 4 : 2;
+  static constexpr int TILE = F8 ? 128 * 128 : 128 * D * 2;
+  static constexpr int QSLOT = F8 ? 128 * D * 2 : TILE;
+  static constexpr int NCH = F8 ? 1 : D / 64;  // 128-byte column chunks of a Q / K row
+  static constexpr int CHUNK = 128 * 128;      // 128 rows x 128 bytes
+  static constexpr int Q_OFF = 0;              // two Q slots (reused as O staging)
+  static constexpr int K_OFF = 2 * QSLOT;
   static constexpr int V_OFF = K_OFF + STAGES * TILE;
   static constexpr int BAR_OFF = V_OFF + STAGES * TILE;
   static constexpr int NBAR = 2 + 6 * STAGES + 8 + 1;
   // d = 64: P gets its own tensor-memory columns (S 128 + P 64 + O 64 per
   // warpgroup fill all 512), so the next QK^T can overwrite S as soon as the
   // softmax has read it; d = 128: P is written over S and waits for PV.
-  static constexpr bool SEP_P = D == 64;
+  static constexpr bool SEP_P = D == 64 && !F8;
   static constexpr uint32_t S_COL = 0;                     // + 128 w
   static constexpr uint32_t P_COL = SEP_P ? 256 : 0;       // + (SEP_P ? 64 : 128) w
   static constexpr uint32_t P_STRIDE = SEP_P ? 64 : 128;
@@ -51,7 +57,8 @@ struct FwdCfg {
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BITS_OFF = MISC_OFF + 64;
   static constexpr int SCHED_OFF = BITS_OFF + 5 * 64 * 4;
-  static constexpr int SMEM_BYTES = SCHED_OFF + kMaxSeg * 4;
+  static constexpr int TMP_OFF = SCHED_OFF + kMaxSeg * 4;  // F8: scratch of the tile reorder
+  static constexpr int SMEM_BYTES = TMP_OFF + (F8 ? kMaxSeg * 4 : 0);
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   // register split: launched at kLaunchRegs per thread, the control
   // warpgroup drops to REGS_CTL and the two softmax warpgroups rise to REGS_SMX
@@ -67,6 +74,7 @@ constexpr bool regs_fit() {
 static_assert(regs_fit<64>() && regs_fit<128>(), "register split exceeds the launch allocation");
 static_assert(FwdCfg<128>::SMEM_ALLOC <= 227 * 1024, "smem budget");
 static_assert(FwdCfg<64>::SMEM_ALLOC <= 227 * 1024, "smem budget");
+static_assert(FwdCfg<128, true>::SMEM_ALLOC <= 227 * 1024, "smem budget");
 
 // Segment entry bits: index in [0, 24), group-valid bits g0..g3 at 24..27, partial at 28.
 constexpr int kGrpShift = 24;
@@ -96,30 +104,6 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // The staged tile may be reused (or the CTA end) once the copies have read
 // it; their global writes complete before the grid does.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// (x0, x1) * c + (o, o), two lanes in one instruction
-__device__ __forceinline__ void fma2(float& x0, float& x1, float c, float o) {
-  uint64_t v, cc, oo;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(x0), "f"(x1));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(cc) : "f"(c));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(oo) : "f"(o));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(v) : "l"(v), "l"(cc), "l"(oo));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(v));
-}
-
-__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
-  uint64_t a, b;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(a) : "f"(a0), "f"(a1));
-  asm("mov.b64 %0, {%1, %2};" : "=l"(b) : "f"(b0), "f"(b1));
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(a) : "l"(a), "l"(b));
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(a));
-}
 
 // Sorted union schedule of the CTA's four 64-row groups (warp 0). Returns count.
 // Warp-parallel throughout: the block-list rows of all groups are read in one
@@ -296,6 +280,56 @@ __device__ __forceinline__ int tile_need(const int32_t* sched, int nseg, int t, 
   return (((g & 3) ? 1 : 0) | ((g & 12) ? 2 : 0)) & act_mask;
 }
 
+// The order in which the CTA walks its full 128-key tiles (F8, four stages):
+// tiles both warpgroups need first, then the tiles of one warpgroup only,
+// alternating between the two while both have some. When the two groups'
+// lists differ, consecutive ring stages then hold tiles of different groups,
+// so neither waits behind a run of the other's tiles. A trailing half tile
+// stays last. Warp-parallel (a rank per class from ballots); `tmp` holds 2n
+// entries.
+__device__ void reorder_tiles(int32_t* sched, int32_t* tmp, int n, int act, int lane) {
+  const int full = n >> 1;
+  if (full < 3) return;
+  int c[4] = {0, 0, 0, 0};
+  for (int t0 = 0; t0 < full; t0 += 32) {
+    const int t = t0 + lane;
+    int cls = -1;
+    if (t < full) {
+      cls = tile_need(sched, n, t, act);
+      if (cls == 0) cls = 3;
+    }
+#pragma unroll
+    for (int k = 1; k < 4; ++k) c[k] += __popc(__ballot_sync(0xffffffffu, cls == k));
+  }
+  const int n3 = c[3], m = min(c[1], c[2]);
+  int base[4] = {0, 0, 0, 0};
+  for (int t0 = 0; t0 < full; t0 += 32) {
+    const int t = t0 + lane;
+    int cls = -1;
+    if (t < full) {
+      cls = tile_need(sched, n, t, act);
+      if (cls == 0) cls = 3;
+    }
+    int pos = 0;
+#pragma unroll
+    for (int k = 1; k < 4; ++k) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, cls == k);
+      if (cls == k) {
+        const int r = base[k] + __popc(bal & ((1u << lane) - 1u));
+        pos = k == 3 ? r : n3 + (r < m ? 2 * r + (k - 1) : 2 * m + (r - m));
+      }
+      base[k] += __popc(bal);
+    }
+    if (t < full) {
+      tmp[2 * pos] = sched[2 * t];
+      tmp[2 * pos + 1] = sched[2 * t + 1];
+    }
+  }
+  __syncwarp();
+  for (int i = lane; i < 2 * full; i += 32) sched[i] = tmp[i];
+  __syncwarp();
+}
+
 // S = Q K^T over D/16 k-steps of 16 (K-major SW128 operands: k-step kk sits
 // in 64-column chunk kk/4 (16 KB apart) at byte offset 32*(kk%4)).
 template <int KK>
@@ -322,6 +356,30 @@ __device__ __forceinline__ void pv_all(uint32_t o_tmem, uint32_t p_tmem, uint64_
   (pv_step<KK>(o_tmem, p_tmem, vd, idesc, first), ...);
 }
 
+// e4m3: S = Q K^T over 4 k-steps of 32 values (32 bytes of the one 128-byte
+// chunk of a row), and O (+)= P V over 4 k-steps of 32 keys: P packed four to
+// a tensor-memory column (8 columns per step), V transposed (K-major, 32 bytes
+// per step).
+template <int KK>
+__device__ __forceinline__ void qk8_step(uint32_t s_tmem, uint64_t qd, uint64_t kd, uint32_t idesc) {
+  umma8_ss_at_warp<KK * 2, KK * 2>(s_tmem, qd, kd, idesc, KK > 0 ? 1u : 0u);
+}
+template <int KK>
+__device__ __forceinline__ void pv8_step(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd, uint32_t idesc,
+                                         uint32_t first) {
+  umma8_ts_at_warp<KK * 8, KK * 2>(o_tmem, p_tmem, vd, idesc, (KK > 0 || !first) ? 1u : 0u);
+}
+template <int... KK>
+__device__ __forceinline__ void qk8_all(uint32_t s_tmem, uint64_t qd, uint64_t kd, uint32_t idesc,
+                                        std::integer_sequence<int, KK...>) {
+  (qk8_step<KK>(s_tmem, qd, kd, idesc), ...);
+}
+template <int... KK>
+__device__ __forceinline__ void pv8_all(uint32_t o_tmem, uint32_t p_tmem, uint64_t vd, uint32_t idesc,
+                                        uint32_t first, std::integer_sequence<int, KK...>) {
+  (pv8_step<KK>(o_tmem, p_tmem, vd, idesc, first), ...);
+}
+
 template <int D>
 __device__ void skip_copy256(const AttnParams& p, int bh, int row0) {
   if (p.cache_in == nullptr) {
@@ -342,12 +400,12 @@ __device__ void skip_copy256(const AttnParams& p, int bh, int row0) {
   }
 }
 
-template <int D>
+template <int D, bool F8 = false>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                const AttnParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, F8>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -415,9 +473,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
     for (int w = 0; w < 2; ++w) {
       mbar_arrive_expect_tx(&q_full[w], C::TILE);
-      for (int c = 0; c < D / 64; ++c)
+      for (int c = 0; c < C::NCH; ++c)
         for (int h2 = 0; h2 < 2; ++h2)
-          tma_load_3d(sQ + w * C::TILE + c * C::CHUNK + h2 * (C::CHUNK / 2), &tmQ, &q_full[w], c * 64,
+          tma_load_3d(sQ + w * C::QSLOT + c * C::CHUNK + h2 * (C::CHUNK / 2), &tmQ, &q_full[w], c * 64,
                       row0 + 128 * w + 64 * h2, bh);
     }
   }
@@ -429,6 +487,7 @@ __global__ void __launch_bounds__(384, 1)
     const int n = build_schedule256(p, mode, bh, row0, vb, vb + 256, sched, lane);
     // tiles each warpgroup needs
     const int act = 1 | ((row0 + 128 < p.N) ? 2 : 0);
+    if constexpr (F8) reorder_tiles(sched, reinterpret_cast<int32_t*>(smem + C::TMP_OFF), n, act, lane);
     const int T = (n + 1) >> 1;
     int c0 = 0, c1 = 0;
     for (int t = lane; t < T; t += 32) {
@@ -446,6 +505,18 @@ __global__ void __launch_bounds__(384, 1)
       misc[3] = c0;
       misc[4] = c1;
       misc[5] = act;
+    }
+  }
+  if constexpr (F8) {
+    // sigma: the head's largest V scale; P is stored as p * sv / sigma, so
+    // every key block's V scale folds into the exponent, and O is scaled by
+    // sigma at the end
+    if (warp == 2) {
+      float m = 0.f;
+      for (int i = lane; i < p.nSeg; i += 32) m = fmaxf(m, __ldg(p.sv + (size_t)bh * p.nSeg + i));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (lane == 0) misc[6] = __float_as_uint(m > 0.f ? m : 1.f);
     }
   }
   tc_fence_before();
@@ -496,7 +567,7 @@ __global__ void __launch_bounds__(384, 1)
         if (t != p.withhold_tile) {
           mbar_arrive_expect_tx(&k_full[st], C::TILE);
           uint8_t* dk = sK + st * C::TILE;
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < C::NCH; ++c) {
             tma_load_3d(dk + c * C::CHUNK, &tmK, &k_full[st], c * 64, sa * 64, bh);
             tma_load_3d(dk + c * C::CHUNK + C::CHUNK / 2, &tmK, &k_full[st], c * 64, sb * 64, bh);
           }
@@ -514,9 +585,18 @@ __global__ void __launch_bounds__(384, 1)
         }
         mbar_arrive_expect_tx(&v_full[st], C::TILE);
         uint8_t* dv = sV + st * C::TILE;
-        for (int c = 0; c < D / 64; ++c) {
-          tma_load_3d(dv + c * C::CHUNK, &tmV, &v_full[st], c * 64, sa * 64, bh);
-          tma_load_3d(dv + c * C::CHUNK + C::CHUNK / 2, &tmV, &v_full[st], c * 64, sb * 64, bh);
+        if constexpr (F8) {
+          // V transposed: the tile's 128 keys are one 128-byte run per channel
+          // row. Key blocks of 128 or more make every tile an aligned pair of
+          // segments (the host checks); anything else is recorded, and the
+          // load still goes out so the pipeline stays whole
+          if ((sa & 1) || (2 * t + 1 < nseg && sb != sa + 1)) record_error(BSA_DEVERR_SCHEDULE);
+          for (int h2 = 0; h2 < 2; ++h2) tma_load_3d(dv + h2 * (C::CHUNK / 2), &tmV, &v_full[st], sa * 64, 64 * h2, bh);
+        } else {
+          for (int c = 0; c < D / 64; ++c) {
+            tma_load_3d(dv + c * C::CHUNK, &tmV, &v_full[st], c * 64, sa * 64, bh);
+            tma_load_3d(dv + c * C::CHUNK + C::CHUNK / 2, &tmV, &v_full[st], c * 64, sb * 64, bh);
+          }
         }
         v_issued = t + 1;
       }
@@ -595,7 +675,7 @@ __global__ void __launch_bounds__(384, 1)
           while (k_seen <= t && ready(&k_full[k_seen % S], (uint32_t)(k_seen / S) & 1u)) ++k_seen;
           if (k_seen <= t) return false;
           tc_fence_after();
-          qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::TILE, 16, 1024),
+          qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::QSLOT, 16, 1024),
                  smem_desc_sw128(sKa + st * C::TILE, 16, 1024), idesc_qk, std::make_integer_sequence<int, D / 16>{});
           tc_commit_warp(&s_full[w]);
           tc_commit_warp(&k_empty[2 * st + w]);
@@ -652,8 +732,8 @@ __global__ void __launch_bounds__(384, 1)
       // so its state and the operand descriptors are warp-uniform; one
       // elected lane issues each MMA and commit.
       if (T > 0) {
-        constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, false, true);
+        constexpr uint32_t idesc_qk = F8 ? idesc_e4m3_f32(128, 128) : idesc_bf16_f32(128, 128, false, false);
+        constexpr uint32_t idesc_pv = F8 ? idesc_e4m3_f32(128, D) : idesc_bf16_f32(128, D, false, true);
         const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
         auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
           return warp_all(mbar_wait(bar, parity, abort_flag, p.wait_limit_ns));
@@ -673,9 +753,14 @@ __global__ void __launch_bounds__(384, 1)
             if (!wwait(&v_full[v_seen % S], (uint32_t)(v_seen / S) & 1u)) return false;
           if (!wwait(&p_full[w], (uint32_t)jj & 1u)) return false;
           tc_fence_after();
-          pv_all(tmem + C::O_COL + w * D, tmem + C::P_COL + w * C::P_STRIDE,
-                 smem_desc_sw128(sVa + (u % S) * C::TILE, C::CHUNK, 1024), idesc_pv, jj == 0 ? 1u : 0u,
-                 std::make_integer_sequence<int, 8>{});
+          if constexpr (F8)
+            pv8_all(tmem + C::O_COL + w * D, tmem + C::P_COL + w * C::P_STRIDE,
+                    smem_desc_sw128(sVa + (u % S) * C::TILE, 16, 1024), idesc_pv, jj == 0 ? 1u : 0u,
+                    std::make_integer_sequence<int, 4>{});
+          else
+            pv_all(tmem + C::O_COL + w * D, tmem + C::P_COL + w * C::P_STRIDE,
+                   smem_desc_sw128(sVa + (u % S) * C::TILE, C::CHUNK, 1024), idesc_pv, jj == 0 ? 1u : 0u,
+                   std::make_integer_sequence<int, 8>{});
           tc_commit_warp(&o_ready[w]);
           tc_commit_warp(&v_empty[2 * (u % S) + w]);
           (w ? pt1 : pt0) = -1;
@@ -691,9 +776,14 @@ __global__ void __launch_bounds__(384, 1)
           // tensor pipe keeps issue order)
           if ((w ? pt1 : pt0) >= 0 && !pv(w)) return false;
           tc_fence_after();
-          qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::TILE, 16, 1024),
-                 smem_desc_sw128(sKa + (t % S) * C::TILE, 16, 1024), idesc_qk,
-                 std::make_integer_sequence<int, D / 16>{});
+          if constexpr (F8)
+            qk8_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::QSLOT, 16, 1024),
+                    smem_desc_sw128(sKa + (t % S) * C::TILE, 16, 1024), idesc_qk,
+                    std::make_integer_sequence<int, 4>{});
+          else
+            qk_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::QSLOT, 16, 1024),
+                   smem_desc_sw128(sKa + (t % S) * C::TILE, 16, 1024), idesc_qk,
+                   std::make_integer_sequence<int, D / 16>{});
           tc_commit_warp(&s_full[w]);
           tc_commit_warp(&k_empty[2 * (t % S) + w]);
           return true;
@@ -755,6 +845,13 @@ __global__ void __launch_bounds__(384, 1)
     const QWin qw = gna_query_window(p.g, pq, p.has_gna && mode == BSA_HEAD_SPARSE);
 
     const float cscale = p.scale_log2;
+    // F8: the row's Q scale, and sigma (the head's largest V scale, from warp 2)
+    float sigma = 1.f, rsig = 1.f, sq_row = 1.f;
+    if constexpr (F8) {
+      sigma = __uint_as_float(misc[6]);
+      rsig = 1.f / sigma;
+      sq_row = __ldg(p.sq + (size_t)bh * p.nSeg + (row_valid ? pq : p.N - 1) / 64);
+    }
     float m = kNegInf, l = 0.f;
     int j = 0;
     bool ok = true;
@@ -816,8 +913,18 @@ __global__ void __launch_bounds__(384, 1)
       }
       xa = fmaxf(xa, sv[63]);
       xb = fmaxf(xb, sv[127]);
-      const float ta = (xa == kNegInf) ? kNegInf : fmaf(xa, cscale, ba);
-      const float tb = (xb == kNegInf) ? kNegInf : fmaf(xb, cscale, bb);
+      // F8: each 64-key half has its own K and V scale; the logit scale takes
+      // sq * sk and the exponent offset log2(sv / sigma), so P holds p * sv / sigma
+      float csa = cscale, csb = cscale, lva = 0.f, lvb = 0.f;
+      if constexpr (F8) {
+        const size_t s0 = (size_t)bh * p.nSeg;
+        csa = cscale * sq_row * __ldg(p.sk + s0 + sa);
+        csb = cscale * sq_row * __ldg(p.sk + s0 + sb);
+        lva = fast_log2(__ldg(p.sv + s0 + sa) * rsig);
+        lvb = fast_log2(__ldg(p.sv + s0 + sb) * rsig);
+      }
+      const float ta = (xa == kNegInf) ? kNegInf : fmaf(xa, csa, ba);
+      const float tb = (xb == kNegInf) ? kNegInf : fmaf(xb, csb, bb);
       const float m_new = max3f(m, ta, tb);
       float alpha = 1.f;
       if (m_new > m + kRescaleTau) {
@@ -825,22 +932,69 @@ __global__ void __launch_bounds__(384, 1)
         m = m_new;
       }
       const float mu = (m == kNegInf) ? 0.f : m;
-      const float oa = ba - mu, ob = bb - mu;
-      // P = exp2(x - m), packed to bf16 in registers first: nothing here
-      // touches tensor memory, so the exps overlap the previous PV
-      float sum0 = 0.f, sum1 = 0.f;
-      uint32_t pk[64];
+      const float oa = ba - mu + lva, ob = bb - mu + lvb;
+      // P = exp2(x - m), packed in registers first: nothing here touches
+      // tensor memory, so the exps overlap the previous PV. bf16: two values
+      // per 32-bit column; F8: four e4m3 codes per column, and the row sum
+      // takes each half's sigma / sv back out.
+      constexpr int NPK = F8 ? 32 : 64;
+      uint32_t pk[NPK];
+      if constexpr (!F8 && !C::SEP_P) {
+        // bf16 over S (d = 128): S(j) landing implies PV(j-1) is complete (its
+        // QK^T was issued after that PV, and a commit tracks every earlier
+        // MMA), so P is written chunk by chunk as it is made, with fewer
+        // registers live than the whole row of P
+        float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float o = i < 32 ? oa : ob;
-        float x0 = sv[2 * i], x1 = sv[2 * i + 1];
-        fma2(x0, x1, cscale, o);
-        x0 = fast_exp2(x0);
-        x1 = fast_exp2(x1);
-        add2(sum0, sum1, x0, x1);
-        pk[i] = pack_bf16x2(x0, x1);
+        for (int c = 0; c < 4; ++c) {
+          const float o = c < 2 ? oa : ob;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0 = sv[32 * c + 2 * i], x1 = sv[32 * c + 2 * i + 1];
+            fma2(x0, x1, cscale, o);
+            x0 = fast_exp2(x0);
+            x1 = fast_exp2(x1);
+            add2(sum0, sum1, x0, x1);
+            pk[16 * c + i] = pack_bf16x2(x0, x1);
+          }
+          tmem_st16(ptm + 16 * c, pk + 16 * c);
+        }
+        l = l * alpha + (sum0 + sum1);
+      } else if constexpr (F8) {
+        float sa0 = 0.f, sa1 = 0.f, sb0 = 0.f, sb1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float o = i < 32 ? oa : ob;
+          const float cs = i < 32 ? csa : csb;
+          float x0 = sv[2 * i], x1 = sv[2 * i + 1];
+          fma2(x0, x1, cs, o);
+          x0 = fast_exp2(x0);
+          x1 = fast_exp2(x1);
+          if (i < 32)
+            add2(sa0, sa1, x0, x1);
+          else
+            add2(sb0, sb1, x0, x1);
+          const uint32_t hw = e4m3x2(x0, x1);
+          if (i & 1)
+            pk[i >> 1] |= hw << 16;
+          else
+            pk[i >> 1] = hw;
+        }
+        l = l * alpha + (sa0 + sa1) * fast_exp2(-lva) + (sb0 + sb1) * fast_exp2(-lvb);
+      } else {
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float o = i < 32 ? oa : ob;
+          float x0 = sv[2 * i], x1 = sv[2 * i + 1];
+          fma2(x0, x1, cscale, o);
+          x0 = fast_exp2(x0);
+          x1 = fast_exp2(x1);
+          add2(sum0, sum1, x0, x1);
+          pk[i] = pack_bf16x2(x0, x1);
+        }
+        l = l * alpha + (sum0 + sum1);
       }
-      l = l * alpha + (sum0 + sum1);
       // PV(j-1) must be complete before P is written (own P columns at d = 64,
       // over S at d = 128) and before O is rescaled; O is rescaled once S is
       // dead (fewer live registers), which is safe because PV(j) waits for p_full
@@ -849,17 +1003,20 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
         tc_fence_after();
       }
+      if constexpr (F8 || C::SEP_P) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_st16(ptm + 16 * c, pk + 16 * c);
+        for (int c = 0; c < NPK / 16; ++c) tmem_st16(ptm + 16 * c, pk + 16 * c);
+      }
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(otm + c * 32, o);
+        // 16 columns at a time: few registers live in this rarely taken branch
+#pragma unroll 1
+        for (int c = 0; c < D / 16; ++c) {
+          float o[16];
+          tmem_ld16(otm + c * 16, o);
           tc_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(otm + c * 32, reinterpret_cast<uint32_t*>(o));
+          for (int i = 0; i < 16; ++i) o[i] *= alpha;
+          tmem_st16(otm + c * 16, reinterpret_cast<uint32_t*>(o));
         }
       }
       tc_wait_st();
@@ -880,8 +1037,8 @@ __global__ void __launch_bounds__(384, 1)
       if (!have) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
       tc_fence_after();
     }
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    uint8_t* stage = sQ + w * C::TILE;  // the Q tile is no longer read once O is final
+    const float inv = l > 0.f ? sigma / l : 0.f;
+    uint8_t* stage = sQ + w * C::QSLOT;  // the Q tile is no longer read once O is final
     const size_t obase = ((size_t)bh * p.N + (row_valid ? pq : 0)) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
@@ -927,10 +1084,11 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D>
+template <int D, bool F8>
 static cudaError_t launch_fwd_d(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
-  auto fn = fwd_kernel<D>;
+  using C = FwdCfg<D, F8>;
+  auto fn = fwd_kernel<D, F8>;
   static DeviceOnce once;
   const cudaError_t e = once.run([&]() -> cudaError_t {
     // the register split needs the full launch allocation: a smaller one
@@ -939,17 +1097,22 @@ static cudaError_t launch_fwd_d(const CUtensorMap& q, const CUtensorMap& k, cons
     cudaError_t r = cudaFuncGetAttributes(&fa, fn);
     if (r != cudaSuccess) return r;
     if (fa.numRegs != kLaunchRegs) return cudaErrorInvalidKernelImage;
-    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdCfg<D>::SMEM_ALLOC);
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
   });
   if (e != cudaSuccess) return e;
-  fn<<<grid, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM_ALLOC, stream>>>(q, k, v, o, p);
+  fn<<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(q, k, v, o, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_forward(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
-  if (d == 64) return launch_fwd_d<64>(q, k, v, o, p, grid, stream);
-  return launch_fwd_d<128>(q, k, v, o, p, grid, stream);
+  if (d == 64) return launch_fwd_d<64, false>(q, k, v, o, p, grid, stream);
+  return launch_fwd_d<128, false>(q, k, v, o, p, grid, stream);
+}
+
+cudaError_t launch_forward_fp8(const CUtensorMap& q8, const CUtensorMap& k8, const CUtensorMap& v8t,
+                               const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
+  return launch_fwd_d<128, true>(q8, k8, v8t, o, p, grid, stream);
 }
 
 }  // namespace bsa

@@ -170,10 +170,23 @@ __global__ void __launch_bounds__(192, 1)
         ba = __ldg(p.bias + bias_row + (sa * 64) / p.block_k) * kLog2e;
         if (sb < p.nSeg) bb = __ldg(p.bias + bias_row + (sb * 64) / p.block_k) * kLog2e;
       }
+      // The per-row reductions below run as several independent chains (a
+      // single 128-long chain of dependent max or add instructions would
+      // take longer than the exps themselves).
+      if (KIND == KIND_LSE) {
+        // z = scale * s + bias, per 64-key half
 #pragma unroll
-      for (int j = 0; j < 64; ++j) s[j] = fmaf(s[j], p.scale_log2, ba);
+        for (int j = 0; j < 64; j += 2) fma2(s[j], s[j + 1], p.scale_log2, ba);
 #pragma unroll
-      for (int j = 64; j < 128; ++j) s[j] = fmaf(s[j], p.scale_log2, bb);
+        for (int j = 64; j < 128; j += 2) fma2(s[j], s[j + 1], p.scale_log2, bb);
+      } else {
+        // z - lse in one step: scale * s + (bias - lse)
+        const float oa = ba - lse2, ob = bb - lse2;
+#pragma unroll
+        for (int j = 0; j < 64; j += 2) fma2(s[j], s[j + 1], p.scale_log2, oa);
+#pragma unroll
+        for (int j = 64; j < 128; j += 2) fma2(s[j], s[j + 1], p.scale_log2, ob);
+      }
       if ((t + 1) * 128 > p.N) {  // ragged last tile: keys past N do not exist
         const uint64_t ma = tail_bits(p.N, sa);
         const uint64_t mb = sb < p.nSeg ? tail_bits(p.N, sb) : 0ull;
@@ -183,25 +196,46 @@ __global__ void __launch_bounds__(192, 1)
         for (int j = 0; j < 64; ++j) s[64 + j] = ((mb >> j) & 1ull) ? s[64 + j] : kNegInf;
       }
       if (KIND == KIND_LSE) {
-        float mx = s[0];
+        // row max: four chains of max3 over the 128 values
+        float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
 #pragma unroll
-        for (int j = 1; j < 128; ++j) mx = fmaxf(mx, s[j]);
+        for (int j = 4; j < 124; j += 8) {
+          m0 = max3f(m0, s[j], s[j + 1]);
+          m1 = max3f(m1, s[j + 2], s[j + 3]);
+          m2 = max3f(m2, s[j + 4], s[j + 5]);
+          m3 = max3f(m3, s[j + 6], s[j + 7]);
+        }
+        m0 = max3f(m0, s[124], s[125]);
+        m1 = max3f(m1, s[126], s[127]);
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
         const float m_new = fmaxf(m, mx);
         if (m_new > m) {
           l *= fast_exp2(m - m_new);
           m = m_new;
         }
         const float mu = (m == kNegInf) ? 0.f : m;
-        float sum = 0.f;
+        // sum of exp2(z - m): four accumulators, two per packed add
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 128; ++j) sum += fast_exp2(s[j] - mu);
-        l += sum;
+        for (int j = 0; j < 128; j += 4) {
+          float x0 = s[j], x1 = s[j + 1], x2 = s[j + 2], x3 = s[j + 3];
+          fma2(x0, x1, 1.f, -mu);
+          fma2(x2, x3, 1.f, -mu);
+          add2(a0, a1, fast_exp2(x0), fast_exp2(x1));
+          add2(a2, a3, fast_exp2(x2), fast_exp2(x3));
+        }
+        l += (a0 + a1) + (a2 + a3);
       } else {
-        float suma = 0.f, sumb = 0.f;
+        // block sums of exp2(z - lse) per 64-key half, two packed accumulators each
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 64; ++j) suma += fast_exp2(s[j] - lse2);
-#pragma unroll
-        for (int j = 64; j < 128; ++j) sumb += fast_exp2(s[j] - lse2);
+        for (int j = 0; j < 64; j += 4) {
+          add2(a0, a1, fast_exp2(s[j]), fast_exp2(s[j + 1]));
+          add2(a2, a3, fast_exp2(s[j + 2]), fast_exp2(s[j + 3]));
+          add2(b0, b1, fast_exp2(s[64 + j]), fast_exp2(s[65 + j]));
+          add2(b2, b3, fast_exp2(s[66 + j]), fast_exp2(s[67 + j]));
+        }
+        float suma = (a0 + a1) + (a2 + a3), sumb = (b0 + b1) + (b2 + b3);
         if (!row_valid) suma = sumb = 0.f;
         const int Ja = (sa * 64) / p.block_k, Jb = (sb * 64) / p.block_k;
         if (Ja == Jb) {

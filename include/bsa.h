@@ -217,6 +217,37 @@ int bsa_forward(const bsa_dims* dims, const void* Q, const void* K, const void* 
                 const bsa_gna_geom* gna, const float* cache_in, float* cache_out,
                 const float* block_bias, float scale, void* O, void* stream);
 
+/* bsa_quantize_fp8: the e4m3 operands of bsa_forward_fp8 (jsqmd.com GNA
+ * article, section 2.1, Blackwell adaptation: FP8 for more tensor-core
+ * throughput; the article gives no scheme). Each 64-token block of each
+ * (b, h) of Q, K and V gets one scale s = amax / 448 (1 for an all-zero
+ * block); the code of x is e4m3(fl32(x * r)) with r = fl32(448 / amax), round
+ * to nearest even, saturating at 448.
+ *  Q, K, V: device bf16 [B, H, N, 128].
+ *  q8, k8: device uint8 [B, H, N, 128] (codes, the layout of Q and K).
+ *  v8t: device uint8 [B, H, 128, Nt], V transposed per head, Nt = N rounded
+ *    up to a multiple of 16; columns N..Nt-1 are written as zero.
+ *  sq, sk, sv: device float [B, H, ceil(N / 64)] (the dequantisation scales).
+ *  All caller-owned; every output is overwritten.
+ *  Errors: INVALID_ARG (null or misaligned pointer, bad dims), UNSUPPORTED
+ *  (d != 128, B * H > 65535), CUDA. */
+int bsa_quantize_fp8(const bsa_dims* dims, const void* Q, const void* K, const void* V, uint8_t* q8,
+                     uint8_t* k8, uint8_t* v8t, float* sq, float* sk, float* sv, void* stream);
+
+/* bsa_forward_fp8: bsa_forward on the e4m3 operands of bsa_quantize_fp8 (same
+ * sections as bsa_quantize_fp8): the attention of the dequantised Q, K and V
+ * (code * scale) over the kept blocks, with the tensor-core products on the
+ * e4m3 codes, P rounded to e4m3 (scaled into range: P holds p * sv / sigma,
+ * sigma the head's largest V scale) and fp32 accumulation; O is bf16
+ * [B, H, N, 128]. Arguments as bsa_forward, with q8, k8, v8t, sq, sk, sv in
+ * place of Q, K and V.
+ *  Errors: as bsa_forward, and UNSUPPORTED for d != 128, block_k not a
+ *  multiple of 128, or a GNA tile volume not a multiple of 128. */
+int bsa_forward_fp8(const bsa_dims* dims, const uint8_t* q8, const uint8_t* k8, const uint8_t* v8t,
+                    const float* sq, const float* sk, const float* sv, const bsa_block_list* list,
+                    const int32_t* head_mode, const bsa_gna_geom* gna, const float* cache_in,
+                    float* cache_out, const float* block_bias, float scale, void* O, void* stream);
+
 /* Length of the tile-order sequence for a raster sequence of n_text text
  * tokens plus the GNA grid: text padded to a multiple of the tile volume,
  * plus every (padded) tile. Host only. */

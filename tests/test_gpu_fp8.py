@@ -1,0 +1,179 @@
+"""GPU e4m3 path (bsa_quantize_fp8 + bsa_forward_fp8) against the fp64 oracle.
+
+* The quantiser's codes decide an integer from floating point, so the oracle takes that decision
+  in the kernel's precision (oracle.fp8.quantize_fp32): codes and scales must match bit for bit,
+  bytes in the OCP e4m3 encoding, V transposed with zero padding.
+* The forward is judged against fp64 attention on the oracle's own dequantised operands
+  (oracle.fp8.quantize / dequantize of the bf16 inputs, the fp64 definition), within a bound per
+  element: the kernel rounds each probability to e4m3 (relative error at most 2^-4, half an e4m3
+  step) and O to bf16 (2^-9 relative), so |O - O_ref| <= 2^-4 * attention(|V|) + 2^-8 |O_ref|
+  + 1e-3 (the last term covers e4m3 subnormals of tiny probabilities and the rare straddled code
+  between the fp64 and the kernel's fp32 quantisation), and the mean error stays within the
+  bf16 bar of 5e-3.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import attention as OA
+from oracle import fp8 as OF8
+from oracle import masks as OM
+from oracle import permute as OP
+from parity_util import bsa, f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _dims(shp):
+    return bsa().dims(shp.B, shp.H, shp.N, shp.d, shp.block_q, shp.block_k, shp.n_text)
+
+
+def _quantize(dm, q, k, v):
+    m = bsa()
+    ops = m.Fp8Operands.empty(dm.B, dm.H, dm.N)
+    ops.v8t.fill_(0xAB)  # the padding columns must come back zero
+    m.quantize_fp8(dm, q.cuda(), k.cuda(), v.cuda(), ops)
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    return ops
+
+
+@pytest.mark.parametrize("B,H,N", [(1, 2, 300), (2, 1, 128), (1, 3, 64 * 7 + 5)])
+def test_quantize_codes_scales_and_layout(B, H, N):
+    q, k, v = W.qkv_normal(B, H, N, 128, N)
+    v[:, :, :64] = 0  # an all-zero block: scale 1, codes 0
+    dm = bsa().dims(B, H, N, 128, 128, 128, 0)
+    ops = _quantize(dm, q, k, v)
+    nt = (N + 15) // 16 * 16
+    for b in range(B):
+        for h in range(H):
+            for x, codes, sc in ((q, ops.q8, ops.sq), (k, ops.k8, ops.sk)):
+                c, s = OF8.quantize_fp32(x[b, h].float().numpy())
+                np.testing.assert_array_equal(codes[b, h].cpu().numpy(), OF8.encode_e4m3(c))
+                np.testing.assert_array_equal(sc[b, h].cpu().numpy(), s.astype(np.float32))
+            c, s = OF8.quantize_fp32(v[b, h].float().numpy())
+            vt = ops.v8t[b, h].cpu().numpy()
+            np.testing.assert_array_equal(vt[:, :N], OF8.encode_e4m3(c).T)
+            assert np.all(vt[:, N:nt] == 0)
+            np.testing.assert_array_equal(ops.sv[b, h].cpu().numpy(), s.astype(np.float32))
+            assert float(ops.sv[b, h, 0]) == 1.0
+
+
+def test_quantize_bytes_equal_torch_float8_on_the_grid():
+    """An independent encoder: a block already on the e4m3 grid with amax 448 has r = 1, so its
+    codes are its own values, whose bytes PyTorch's float8_e4m3fn conversion gives."""
+    q, k, v = W.qkv_normal(1, 1, 256, 128, 7)
+    g = torch.from_numpy(np.random.default_rng(7).choice(OF8.e4m3_values(), (64, 128)).astype(np.float32))
+    g[0, 0] = 448.0
+    q[0, 0, 64:128] = g.to(torch.bfloat16)
+    ops = _quantize(bsa().dims(1, 1, 256, 128, 128, 128, 0), q, k, v)
+    assert float(ops.sq[0, 0, 1]) == 1.0
+    ref = q[0, 0, 64:128].float().to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(ops.q8[0, 0, 64:128].cpu().numpy(), ref)
+
+
+def _dequantised(x):
+    """The oracle's operand: fp64 quantise / dequantise of the bf16 values of one (b, h)."""
+    c, s = OF8.quantize(f64(x))
+    return OF8.dequantize(c, s)
+
+
+def _check_rows(got, q, k, v, mode, fn, rows, bias_fn=None, what=""):
+    qd, kd, vd = (_dequantised(t) for t in (q, k, v))
+    exp = OA.head_forward(qd, kd, vd, mode, fn, 128 ** -0.5, rows=rows, bias_fn=bias_fn)
+    bound = OA.head_forward(qd, kd, np.abs(vd), mode, fn, 128 ** -0.5, rows=rows, bias_fn=bias_fn)
+    err = np.abs(got - exp)
+    ok = err <= 2.0 ** -4 * bound + 2.0 ** -8 * np.abs(exp) + 1e-3
+    assert ok.all(), f"{what}: worst {float(err.max()):.3e} at {np.unravel_index(np.argmax(err - bound), err.shape)}"
+    assert err.mean() <= 5e-3, f"{what}: mean {float(err.mean()):.3e}"
+
+
+@pytest.mark.parametrize("N", [128 * 6, 128 * 6 + 40])
+def test_forward_fp8_arrow_full_skip(N):
+    m = bsa()
+    w = W.arrow_case(B=1, H=4, n_text=128, grid_hw=(1, N - 128), d=128, block=128, seed=N,
+                     fracs=(0.25, 0.5, 0.25))
+    shp = w["shape"]
+    dm = _dims(shp)
+    ops = _quantize(dm, w["q"], w["k"], w["v"])
+    modes = torch.from_numpy(w["head_mode"]).cuda()
+    blocks = m.BlockList.empty(1, shp.H, shp.n_qb, shp.n_kb, bitmap=False)
+    m.build_mask(dm, m.MASK_ARROW, blocks, head_mode=modes, window=torch.from_numpy(w["window"]).cuda())
+    o = torch.empty(w["q"].shape, dtype=torch.bfloat16, device="cuda")
+    m.forward_fp8(dm, ops, o, modes, blocks=blocks, cache_in=w["cache"].cuda())
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    for h in range(shp.H):
+        mode = int(w["head_mode"][h])
+        if mode == W.HEAD_SKIP:  # the cache path is the bf16 one: exact
+            exp = OA.bf16_round(w["cache"][0, h].numpy().astype(np.float32))
+            np.testing.assert_array_equal(f64(o[0, h]), exp)
+            continue
+        fn = lambda r, h=h, mode=mode: OM.arrow_token_mask(N, shp.n_text, 128, mode, int(w["window"][h]), r)
+        _check_rows(f64(o[0, h]), w["q"][0, h], w["k"][0, h], w["v"][0, h], mode, fn, np.arange(N), what=f"h{h}")
+
+
+def test_forward_fp8_block_bias_and_peaked_rows():
+    """A block bias and large logits (scaled Q) give peaked rows, where the lazy rescale and the
+    P scaling into e4m3 range matter most."""
+    m = bsa()
+    B, H, N, bs = 1, 2, 128 * 5 + 30, 128
+    q, k, v = W.qkv_normal(B, H, N, 128, 11)
+    q = (q.float() * 3.0).to(torch.bfloat16)
+    nb = -(-N // bs)
+    bias, _ = W.dlm_bias(H, nb, nb - 1, seed=3, n_col_pre=2, n_col_gen=1, windows=(1,))
+    dm = m.dims(B, H, N, 128, bs, bs, 0)
+    ops = _quantize(dm, q, k, v)
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    modes = torch.zeros(H, dtype=torch.int32, device="cuda")
+    m.forward_fp8(dm, ops, o, modes, bias=bias.cuda())
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    for h in range(H):
+        bfn = OA.block_bias_fn(bias[h].numpy(), bs, bs, N)
+        _check_rows(f64(o[0, h]), q[0, h], k[0, h], v[0, h], OM.HEAD_FULL, lambda r: np.ones((len(r), N), bool),
+                    np.arange(N), bias_fn=bfn, what=f"h{h}")
+
+
+@pytest.mark.parametrize("stride", [(1, 1, 1), (2, 4, 4)])
+def test_forward_fp8_gna_partial_tiles(stride):
+    """GNA tiles of 2 x 8 x 8 = 128 tokens in tile order with partial tiles (the fine mask) and a
+    padded grid."""
+    m = bsa()
+    n_text, grid, tile, window = 128, (4, 12, 20), (2, 8, 8), (3, 9, 11)
+    wl = W.video_case(1, 2, n_text, grid, tile, window, stride, 128, 9)
+    lay = OM.GnaLayout(n_text, grid, tile, window, stride)
+    g = m.GnaGeom.make(grid, tile, window, stride)
+    nt = m.gna_tiled_len(n_text, g)
+    dm_r = m.dims(1, 2, wl["shape"].N, 128, lay.bs, lay.bs, n_text)
+    dm = m.dims(1, 2, nt, 128, lay.bs, lay.bs, n_text)
+    raster = [t.cuda() for t in (wl["q"], wl["k"], wl["v"])]
+    tiled = [torch.empty((1, 2, nt, 128), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    m.permute_tiles(dm_r, g, raster, tiled)
+    ops = _quantize(dm, *tiled)
+    nb = nt // lay.bs
+    blocks = m.BlockList.empty(1, 2, nb, nb, bitmap=False)
+    modes = torch.ones(2, dtype=torch.int32, device="cuda")
+    m.build_mask(dm, m.MASK_GNA, blocks, head_mode=modes, gna=g)
+    o = torch.empty_like(tiled[0])
+    m.forward_fp8(dm, ops, o, modes, blocks=blocks, gna=g)
+    torch.cuda.synchronize()
+    assert m.get_device_error() == 0
+    rows = np.nonzero(lay.valid(np.arange(nt)))[0]
+    for h in range(2):
+        qt, kt, vt = (OP.permute_to_tiles(f64(t[0, h]), lay) for t in (wl["q"], wl["k"], wl["v"]))
+        _check_rows(f64(o[0, h])[rows], torch.from_numpy(qt), torch.from_numpy(kt), torch.from_numpy(vt),
+                    OM.HEAD_SPARSE, lambda r: OM.gna_token_mask(lay, r), rows, what=f"gna h{h}")
+
+
+def test_fp8_rejects_what_it_does_not_cover():
+    m = bsa()
+    q = torch.zeros(1, 1, 256, 64, dtype=torch.bfloat16, device="cuda")
+    ops = m.Fp8Operands.empty(1, 1, 256, 64)
+    with pytest.raises(m.BsaError):  # d = 64
+        m.quantize_fp8(m.dims(1, 1, 256, 64, 64, 64, 0), q, q, q, ops)
+    ops = m.Fp8Operands.empty(1, 1, 256)
+    o = torch.empty(1, 1, 256, 128, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(m.BsaError):  # key blocks of 64
+        m.forward_fp8(m.dims(1, 1, 256, 128, 64, 64, 0), ops, o, torch.zeros(1, dtype=torch.int32, device="cuda"))
