@@ -53,6 +53,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 forward leg (d = 128 workloads)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="oracle sample budget")
     ap.add_argument("--shard", default="replicas", choices=["replicas", "heads"],
                     help="N > 1: independent replicas per GPU (weak scaling, default), or one problem split "
@@ -278,6 +279,10 @@ class ContentJob(Job):
     def e2e_output(self):
         return self.o
 
+    def fwd_args(self):
+        """(dims, Q, K, V, head modes, keyword arguments) of this step's forward."""
+        return self.dm, self.q, self.k, self.v, self.modes, {"blocks": self.blocks}
+
     def phases(self):
         """The HBM-bound steps, each with its algorithmic bytes: pooling reads Q and K once."""
         bsa, s = self.bsa, self.s
@@ -342,6 +347,10 @@ class DlmJob(Job):
     def e2e_output(self):
         return self.o
 
+    def fwd_args(self):
+        q, k, v = self.sets[0]
+        return self.dm, q, k, v, self.modes, {"blocks": self.blocks, "bias": self.bias}
+
     def step(self, ev_fwd=None):
         q, k, v = self.sets[self.i % len(self.sets)]
         self.i += 1
@@ -386,6 +395,10 @@ class VideoJob(Job):
 
     def e2e_output(self):
         return self.o
+
+    def fwd_args(self):
+        return self.dm, self.tiled[0], self.tiled[1], self.tiled[2], self.modes, {"blocks": self.blocks,
+                                                                                    "gna": self.geom}
 
     def phases(self):
         """The HBM-bound steps, each with its algorithmic bytes (every row read once, written once)."""
@@ -534,6 +547,41 @@ def gna_useful_pairs(n_text, grid, window):
         n_img *= L
         win *= min(k, L)
     return n_img * (win + n_text) + n_text * (n_text + n_img)
+
+
+def fp8_leg(job, flush, bf16_peak, reps=20, warmup=3):
+    """The e4m3 forward (bsa_quantize_fp8 + bsa_forward_fp8) on the operands and block list of the
+    job's bf16 forward: the quantisation and the forward each timed alone (CUDA events, L2
+    flushed before every call, median of `reps`). Its roofline peak is the measured bf16 peak
+    times the nominal 2x of e4m3 over bf16 dense tensor throughput."""
+    bsa = job.bsa
+    dm, q, k, v, modes, kw = job.fwd_args()
+    ops = bsa.Fp8Operands.empty(dm.B, dm.H, dm.N)
+    o = torch.empty_like(q)
+
+    def timed(fn):
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for e0, e1 in evs:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return float(np.median([e0.elapsed_time(e1) for e0, e1 in evs]))
+    q_ms = timed(lambda: bsa.quantize_fp8(dm, q, k, v, ops))
+    f_ms = timed(lambda: bsa.forward_fp8(dm, ops, o, modes, **kw))
+    if bsa.get_device_error() != 0:
+        raise RuntimeError("device error in the e4m3 forward")
+    achieved = job.flops / (f_ms * 1e-3) / 1e12
+    peak = 2.0 * bf16_peak
+    return {"fwd_ms": f_ms, "fwd_tflops": achieved, "quantize_ms": q_ms,
+            "step_tflops_with_quantize": job.flops / ((f_ms + q_ms) * 1e-3) / 1e12,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "kernel": "bsa::fwd_kernel<128, true> (bsa_forward_fp8)",
+                         "peak_source": "measured bf16 burst x 2 (nominal e4m3 / bf16 dense ratio)"}}
 
 
 def phase_bandwidth(phases, flush, hbm_gbs, reps=20, warmup=3):
@@ -828,6 +876,8 @@ def run_bsa(args, rank, world, local_rank):
     if hasattr(inner, "useful_flops"):  # pairs the mask allows, partial tiles counted by their real pairs
         extra["useful_tflops"] = inner.useful_flops / (fwd_ms_mean * 1e-3) / 1e12
         extra["useful_flops_per_step"] = inner.useful_flops
+    if not args.no_fp8 and hasattr(inner, "fwd_args") and inner.s.d == 128:
+        extra["fp8"] = fp8_leg(inner, flush, peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     if hasattr(inner, "phases"):
         hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
         extra["hbm_phases"] = phase_bandwidth(inner.phases(), flush, hbm)

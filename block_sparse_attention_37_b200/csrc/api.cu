@@ -118,8 +118,13 @@ int make_gna(const bsa_gna_geom* in, int n_text, GnaDev* g) {
   const int tx = g->tile[2];
   g->seg_one_slice = tx <= 64 && 64 % tx == 0 && g->tile[1] % (64 / tx) == 0;
   g->x_rep = 0ull;
-  if (g->seg_one_slice)
-    for (int r = 0; r < 64 / tx; ++r) g->x_rep |= 1ull << (tx * r);
+  g->seg_rows = 0;
+  g->x_mask = 0ull;
+  if (g->seg_one_slice) {
+    g->seg_rows = 64 / tx;
+    for (int r = 0; r < g->seg_rows; ++r) g->x_rep |= 1ull << (tx * r);
+    g->x_mask = tx >= 64 ? ~0ull : ((1ull << tx) - 1ull);
+  }
   g->has_padding = g->text_span > n_text;
   for (int d = 0; d < 3; ++d) g->has_padding |= (g->grid[d] % g->tile[d]) != 0;
   return BSA_OK;

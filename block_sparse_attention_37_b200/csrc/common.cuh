@@ -422,6 +422,8 @@ struct GnaDev {
   // and cut to the row range
   int seg_one_slice;
   uint64_t x_rep;
+  int seg_rows;     // 64 / x-extent: rows of the tile in one segment (one-slice layouts)
+  uint64_t x_mask;  // bits [0, x-extent)
 };
 
 __host__ __device__ __forceinline__ int gna_window_start(int i, int L, int k, int s) {

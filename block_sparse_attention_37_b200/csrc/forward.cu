@@ -58,7 +58,8 @@ struct FwdCfg {
   static constexpr int BITS_OFF = MISC_OFF + 64;
   static constexpr int SCHED_OFF = BITS_OFF + 5 * 64 * 4;
   static constexpr int TMP_OFF = SCHED_OFF + kMaxSeg * 4;  // F8: scratch of the tile reorder
-  static constexpr int SMEM_BYTES = TMP_OFF + (F8 ? kMaxSeg * 4 : 0);
+  static constexpr int GEO_OFF = TMP_OFF + (F8 ? kMaxSeg * 4 : 0);  // segment geometry (GNA)
+  static constexpr int SMEM_BYTES = GEO_OFF + kMaxSeg * 8;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   // register split: launched at kLaunchRegs per thread, the control
   // warpgroup drops to REGS_CTL and the two softmax warpgroups rise to REGS_SMX
@@ -75,6 +76,7 @@ static_assert(regs_fit<64>() && regs_fit<128>(), "register split exceeds the lau
 static_assert(FwdCfg<128>::SMEM_ALLOC <= 227 * 1024, "smem budget");
 static_assert(FwdCfg<64>::SMEM_ALLOC <= 227 * 1024, "smem budget");
 static_assert(FwdCfg<128, true>::SMEM_ALLOC <= 227 * 1024, "smem budget");
+static_assert(FwdCfg<64, false>::SMEM_ALLOC <= 227 * 1024 && FwdCfg<128, false>::SMEM_ALLOC <= 227 * 1024, "smem budget");
 
 // Segment entry bits: index in [0, 24), group-valid bits g0..g3 at 24..27, partial at 28.
 constexpr int kGrpShift = 24;
@@ -488,6 +490,14 @@ __global__ void __launch_bounds__(384, 1)
     // tiles each warpgroup needs
     const int act = 1 | ((row0 + 128 < p.N) ? 2 : 0);
     if constexpr (F8) reorder_tiles(sched, reinterpret_cast<int32_t*>(smem + C::TMP_OFF), n, act, lane);
+    // where every partial segment sits in the grid, once for the whole CTA
+    if (p.has_gna && p.g.seg_one_slice) {
+      uint64_t* geo = reinterpret_cast<uint64_t*>(smem + C::GEO_OFF);
+      for (int i = lane; i < n; i += 32) {
+        const int e = sched[i];
+        if (e & kPart4) geo[i] = gna_segment_geo(p.g, e & kSegIdxMask);
+      }
+    }
     const int T = (n + 1) >> 1;
     int c0 = 0, c1 = 0;
     for (int t = lane; t < T; t += 32) {
@@ -843,6 +853,9 @@ __global__ void __launch_bounds__(384, 1)
     const int my_bit = 1 << (kGrpShift + grp);
 
     const QWin qw = gna_query_window(p.g, pq, p.has_gna && mode == BSA_HEAD_SPARSE);
+    const QBox qb = gna_query_box(p.g, qw);
+    const bool geo_fast = p.has_gna && p.g.seg_one_slice;
+    const uint64_t* geo = reinterpret_cast<const uint64_t*>(smem + C::GEO_OFF);
 
     const float cscale = p.scale_log2;
     // F8: the row's Q scale, and sigma (the head's largest V scale, from warp 2)
@@ -878,11 +891,13 @@ __global__ void __launch_bounds__(384, 1)
         mb = 0ull;
         if (ea & my_bit) {
           ma = tail_bits(p.N, sa);
-          if ((ea & kPart4) && p.has_gna) ma &= gna_segment_bits(p.g, sa, qw);
+          if ((ea & kPart4) && p.has_gna)
+            ma &= geo_fast ? gna_segment_bits_geo(p.g, sa, geo[2 * t], qb) : gna_segment_bits(p.g, sa, qw);
         }
         if (eb >= 0 && (eb & my_bit)) {
           mb = tail_bits(p.N, sb);
-          if ((eb & kPart4) && p.has_gna) mb &= gna_segment_bits(p.g, sb, qw);
+          if ((eb & kPart4) && p.has_gna)
+            mb &= geo_fast ? gna_segment_bits_geo(p.g, sb, geo[2 * t + 1], qb) : gna_segment_bits(p.g, sb, qw);
         }
       }
       // The whole 128-key row of S is read once into registers: with its own
@@ -903,16 +918,19 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < 64; ++i) sv[64 + i] = ((mb >> i) & 1ull) ? sv[64 + i] : kNegInf;
       }
-      // row max of the raw scores, per 64-key half (the bias is constant per half)
-      float xa = max3f(sv[0], sv[1], sv[2]);
-      float xb = max3f(sv[64], sv[65], sv[66]);
+      // row max of the raw scores, per 64-key half (the bias is constant per
+      // half): two independent max3 chains per half
+      float xa0 = max3f(sv[0], sv[1], sv[2]), xa1 = max3f(sv[3], sv[4], sv[5]);
+      float xb0 = max3f(sv[64], sv[65], sv[66]), xb1 = max3f(sv[67], sv[68], sv[69]);
 #pragma unroll
-      for (int i = 3; i < 63; i += 2) {
-        xa = max3f(xa, sv[i], sv[i + 1]);
-        xb = max3f(xb, sv[64 + i], sv[65 + i]);
+      for (int i = 6; i < 62; i += 4) {
+        xa0 = max3f(xa0, sv[i], sv[i + 1]);
+        xa1 = max3f(xa1, sv[i + 2], sv[i + 3]);
+        xb0 = max3f(xb0, sv[64 + i], sv[65 + i]);
+        xb1 = max3f(xb1, sv[66 + i], sv[67 + i]);
       }
-      xa = fmaxf(xa, sv[63]);
-      xb = fmaxf(xb, sv[127]);
+      const float xa = max3f(xa0, xa1, fmaxf(sv[62], sv[63]));
+      const float xb = max3f(xb0, xb1, fmaxf(sv[126], sv[127]));
       // F8: each 64-key half has its own K and V scale; the logit scale takes
       // sq * sk and the exponent offset log2(sv / sigma), so P holds p * sv / sigma
       float csa = cscale, csb = cscale, lva = 0.f, lvb = 0.f;

@@ -70,12 +70,16 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(QuantParams p) {
   if (threadIdx.x == 0) (t == 0 ? p.sq : p.sk)[bh * p.nS + blk] = m > 0.f ? m / 448.f : 1.f;
 }
 
+// Row pitch of the staged V codes: a multiple of 8 (every key row is written with 8-byte
+// stores) that is not a multiple of 128, so the column reads of the transpose spread over banks.
+constexpr int kStPitch = 136;
+
 // V: one CTA per (128-key tile, b*h). The tile's two 64-key blocks are scaled on their own,
-// staged as codes [key][channel] (row pitch 132 bytes against bank conflicts), then written
-// transposed: channel c's 128 codes of the tile are one contiguous 128-byte run of v8t
+// staged as codes [key][channel] (row pitch kStPitch), then written transposed: channel c's 128
+// codes of the tile are one contiguous 128-byte run of v8t
 __global__ void __launch_bounds__(256) quant_vt_kernel(QuantParams p) {
   __shared__ float red[8];
-  __shared__ __align__(16) uint8_t st[128 * 132];
+  __shared__ __align__(16) uint8_t st[128 * kStPitch];
   const int tile = blockIdx.x;
   const long long bh = blockIdx.y;
   const int key0 = tile * 128;
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(256) quant_vt_kernel(QuantParams p) {
     for (int u = 0; u < 4; ++u) {
       const int i = threadIdx.x + 256 * u;
       const int key = half * 64 + (i >> 4);
-      *reinterpret_cast<uint2*>(st + key * 132 + (i & 15) * 8) = codes8(v[u], r);
+      *reinterpret_cast<uint2*>(st + key * kStPitch + (i & 15) * 8) = codes8(v[u], r);
     }
     if (threadIdx.x == 0 && tile * 2 + half < p.nS) p.sv[bh * p.nS + tile * 2 + half] = m > 0.f ? m / 448.f : 1.f;
     __syncthreads();  // red[] is reused by the second half; st[] is read below
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(256) quant_vt_kernel(QuantParams p) {
     for (int q = 0; q < 4; ++q) {
       uint32_t x = 0;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) x |= (uint32_t)st[(g * 16 + q * 4 + b) * 132 + c] << (8 * b);
+      for (int b = 0; b < 4; ++b) x |= (uint32_t)st[(g * 16 + q * 4 + b) * kStPitch + c] << (8 * b);
       w[q] = x;
     }
     // Nt is a multiple of 16 and k0 a multiple of 16: the 16 bytes stay inside the row

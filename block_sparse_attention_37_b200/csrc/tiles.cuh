@@ -168,4 +168,64 @@ __host__ __device__ __forceinline__ uint64_t gna_segment_bits(const GnaDev& g, i
   return m;
 }
 
+// Precomputed segment geometry (one-slice layouts). The forward computes,
+// once per CTA while it builds the key schedule, where each partial 64-key
+// segment sits in the grid: the t, y and x of its first key (17 bits each;
+// a sequence of at most 131072 tokens keeps every coordinate below 2^17). A
+// text segment is marked instead and keeps the text rule. Each softmax
+// thread then needs only a few compares per segment against its query's
+// clamped window (QBox), computed once before the tile loop.
+constexpr uint64_t kGeoText = 1ull << 63;
+
+__host__ __device__ inline uint64_t gna_segment_geo(const GnaDev& g, int seg) {
+  const int k0 = seg * 64;
+  if (k0 < g.text_span) return kGeoText;
+  const int v0 = k0 - g.text_span;
+  const int tile = fdiv(v0, g.f_vol);
+  const int l0 = v0 - tile * g.vol;
+  const int q2 = fdiv(tile, g.f_tiles2);
+  const int tx = tile - q2 * g.tiles[2];
+  const int tt = fdiv(q2, g.f_tiles1);
+  const int ty = q2 - tt * g.tiles[1];
+  const int R0 = fdiv(l0, g.f_tile2);
+  const int tq = fdiv(R0, g.f_tile1);
+  const int t = tt * g.tile[0] + tq;
+  const int y0 = ty * g.tile[1] + (R0 - tq * g.tile[1]);
+  const int x0 = tx * g.tile[2];
+  return (uint64_t)t | ((uint64_t)y0 << 17) | ((uint64_t)x0 << 34);
+}
+
+struct QBox {
+  int tlo, thi, ylo, yhi, xlo, xhi;
+};
+
+// A query's window clamped to the grid (padding keys fall outside it).
+__host__ __device__ inline QBox gna_query_box(const GnaDev& g, const QWin& q) {
+  QBox b;
+  b.tlo = q.lo0 > 0 ? q.lo0 : 0;
+  b.thi = q.hi0 < g.grid[0] ? q.hi0 : g.grid[0];
+  b.ylo = q.lo1 > 0 ? q.lo1 : 0;
+  b.yhi = q.hi1 < g.grid[1] ? q.hi1 : g.grid[1];
+  b.xlo = q.lo2 > 0 ? q.lo2 : 0;
+  b.xhi = q.hi2 < g.grid[2] ? q.hi2 : g.grid[2];
+  return b;
+}
+
+// gna_segment_bits for a one-slice layout from the precomputed geometry.
+__host__ __device__ __forceinline__ uint64_t gna_segment_bits_geo(const GnaDev& g, int seg, uint64_t geo,
+                                                                  const QBox& b) {
+  if (geo & kGeoText) {
+    const int nt = g.n_text - seg * 64;
+    return nt <= 0 ? 0ull : (nt >= 64 ? ~0ull : ((1ull << nt) - 1ull));
+  }
+  const int t = (int)(geo & 0x1FFFFull), y0 = (int)((geo >> 17) & 0x1FFFFull), x0 = (int)((geo >> 34) & 0x1FFFFull);
+  if (t < b.tlo || t >= b.thi) return 0ull;
+  const int rlo = b.ylo - y0 > 0 ? b.ylo - y0 : 0;
+  const int rhi = b.yhi - y0 < g.seg_rows ? b.yhi - y0 : g.seg_rows;
+  if (rlo >= rhi) return 0ull;
+  const int Tx = g.tile[2];
+  const uint64_t xb = bit_range64(b.xlo - x0, b.xhi - x0) & g.x_mask;
+  return (xb * g.x_rep) & bit_range64(rlo * Tx, rhi * Tx);
+}
+
 }  // namespace bsa

@@ -32,6 +32,15 @@ extern "C" int h_segbits_row(int n_text, const bsa_gna_geom* geom, int pq, unsig
   for (int s = 0; s < nseg; ++s) out[s] = bsa::gna_segment_bits(g, s, q);
   return 0;
 }
+extern "C" int h_segbits_geo_row(int n_text, const bsa_gna_geom* geom, int pq, unsigned long long* out, int nseg) {
+  bsa::GnaDev g;
+  const int st = bsa::make_gna(geom, n_text, &g);
+  if (st) return st;
+  if (!g.seg_one_slice) return -1;
+  const bsa::QBox b = bsa::gna_query_box(g, bsa::gna_query_window(g, pq, true));
+  for (int s = 0; s < nseg; ++s) out[s] = bsa::gna_segment_bits_geo(g, s, bsa::gna_segment_geo(g, s), b);
+  return 0;
+}
 extern "C" int h_gna_classes(int n_text, const bsa_gna_geom* geom, unsigned char* out, int nb) {
   bsa::GnaDev g;
   const int st = bsa::make_gna(geom, n_text, &g);
@@ -72,6 +81,7 @@ def host_lib(tmp_path_factory):
     lib.h_tile_sources.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.h_gna_classes.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.h_fdiv_many.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+    lib.h_segbits_geo_row.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
     return lib
 
 
@@ -131,6 +141,30 @@ def test_fine_mask_bits_equal_the_token_mask(host_lib, n_text, grid, tile, windo
     shifts = np.arange(64, dtype=np.uint64)
     for pq in rows:
         assert host_lib.h_segbits_row(n_text, ctypes.byref(g), int(pq), out.ctypes.data, nseg) == 0
+        got = ((out[:, None] >> shifts[None, :]) & np.uint64(1)).astype(bool).reshape(-1)[:lay.N]
+        exp = OM.gna_token_mask(lay, [int(pq)])[0]
+        assert np.array_equal(got, exp), (grid, int(pq), np.nonzero(got != exp)[0][:5])
+
+
+@pytest.mark.parametrize("n_text,grid,tile,window,stride", CASES)
+def test_precomputed_geometry_bits_equal_the_token_mask(host_lib, n_text, grid, tile, window, stride):
+    """The forward's fast path for layouts whose segments lie in one t-slice: the segment's grid
+    position computed once (schedule build) and each query's clamped window once give the same
+    bits as the token mask."""
+    lay = OM.GnaLayout(n_text, grid, tile, window, stride)
+    g = _geom(grid, tile, window, stride)
+    nseg = -(-lay.N // 64)
+    rows = np.arange(lay.N)
+    if lay.N > 4096:
+        rows = np.sort(np.random.default_rng(lay.N + 1).choice(lay.N, 256, replace=False))
+    rows = rows[lay.valid(rows)]
+    out = np.zeros(nseg, dtype=np.uint64)
+    shifts = np.arange(64, dtype=np.uint64)
+    for pq in rows:
+        st = host_lib.h_segbits_geo_row(n_text, ctypes.byref(g), int(pq), out.ctypes.data, nseg)
+        if st == -1:
+            pytest.skip("segments span several t-slices: the forward keeps the general path")
+        assert st == 0
         got = ((out[:, None] >> shifts[None, :]) & np.uint64(1)).astype(bool).reshape(-1)[:lay.N]
         exp = OM.gna_token_mask(lay, [int(pq)])[0]
         assert np.array_equal(got, exp), (grid, int(pq), np.nonzero(got != exp)[0][:5])
