@@ -16,9 +16,12 @@
 
 namespace bsa {
 
+// Two CTAs per SM (96 KB of shared memory and 256 tensor-memory columns
+// each at d = 128): each scheduler then runs two row warps, whose exps and
+// reductions hide each other's latency.
 template <int D>
 struct ScoreCfg {
-  static constexpr int STAGES = D == 64 ? 4 : 3;
+  static constexpr int STAGES = D == 64 ? 4 : 2;
   static constexpr int TILE_BYTES = 128 * D * 2;
   static constexpr int CHUNK_BYTES = 128 * 128;
   static constexpr int Q_OFF = 0;
@@ -30,10 +33,11 @@ struct ScoreCfg {
   static constexpr int SMEM_BYTES = MISC_OFF + 64;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 };
-static_assert(ScoreCfg<128>::SMEM_ALLOC <= 227 * 1024, "smem budget");
+static_assert(2 * ScoreCfg<128>::SMEM_ALLOC <= 227 * 1024 && 2 * ScoreCfg<64>::SMEM_ALLOC <= 227 * 1024,
+              "two CTAs per SM");
 
 template <int D, int KIND>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, 2)
     score_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const AttnParams p) {
   using C = ScoreCfg<D>;

@@ -66,7 +66,6 @@ __device__ __forceinline__ float sanitize(float x) { return (x == x) ? x : -__in
 template <int D>
 __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
   extern __shared__ float sc[];  // [nKB] scores
-  __shared__ float qv[D];
   __shared__ int warp_tot[8];
   uint8_t* keep = reinterpret_cast<uint8_t*>(sc + p.nKB);
   const int I = blockIdx.x % p.nQB;
@@ -75,21 +74,41 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (p.method == BSA_SELECT_POOLED_QK) {
-    for (int j = tid; j < D; j += 256) qv[j] = p.qbar[row * D + j];
-    __syncthreads();
+    // One warp per key block: the lanes read the pooled key row together
+    // (D / 32 consecutive floats each, one coalesced row per load) and
+    // reduce the dot product with shuffles.
+    constexpr int PL = D / 32;  // floats per lane
+    float qr[PL];
+#pragma unroll
+    for (int i = 0; i < PL; ++i) qr[i] = p.qbar[row * D + lane * PL + i];
     const float* kb = p.kbar + (size_t)bh * p.nKB * D;
-    for (int J = tid; J < p.nKB; J += 256) {
-      const float4* kr = reinterpret_cast<const float4*>(kb + (size_t)J * D);
-      float s = 0.f;
-#pragma unroll 8
-      for (int j = 0; j < D / 4; ++j) {
-        const float4 k4 = __ldg(kr + j);
-        s = fmaf(qv[4 * j], k4.x, s);
-        s = fmaf(qv[4 * j + 1], k4.y, s);
-        s = fmaf(qv[4 * j + 2], k4.z, s);
-        s = fmaf(qv[4 * j + 3], k4.w, s);
+    // eight key rows per warp in flight at a time (their loads are
+    // independent), then the eight reductions
+    constexpr int R = 8;
+    for (int J0 = warp; J0 < p.nKB; J0 += 8 * R) {
+      float kv[R][PL];
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int J = J0 + 8 * r;
+        const float* kr = kb + (size_t)(J < p.nKB ? J : 0) * D + lane * PL;
+        if constexpr (PL == 4) {
+          const float4 k4 = __ldg(reinterpret_cast<const float4*>(kr));
+          kv[r][0] = k4.x; kv[r][1] = k4.y; kv[r][2] = k4.z; kv[r][3] = k4.w;
+        } else {
+          const float2 k2 = __ldg(reinterpret_cast<const float2*>(kr));
+          kv[r][0] = k2.x; kv[r][1] = k2.y;
+        }
       }
-      sc[J] = sanitize(s);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = PL - 1; i >= 0; --i) s = fmaf(qr[i], kv[r][i], s);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        const int J = J0 + 8 * r;
+        if (lane == 0 && J < p.nKB) sc[J] = sanitize(s);
+      }
     }
   } else {
     const int nq = min(p.block_q, p.N - I * p.block_q);

@@ -3,13 +3,20 @@
 * The quantiser's codes decide an integer from floating point, so the oracle takes that decision
   in the kernel's precision (oracle.fp8.quantize_fp32): codes and scales must match bit for bit,
   bytes in the OCP e4m3 encoding, V transposed with zero padding.
-* The forward is judged against fp64 attention on the oracle's own dequantised operands
-  (oracle.fp8.quantize / dequantize of the bf16 inputs, the fp64 definition), within a bound per
-  element: the kernel rounds each probability to e4m3 (relative error at most 2^-4, half an e4m3
-  step) and O to bf16 (2^-9 relative), so |O - O_ref| <= 2^-4 * attention(|V|) + 2^-8 |O_ref|
-  + 1e-3 (the last term covers e4m3 subnormals of tiny probabilities and the rare straddled code
-  between the fp64 and the kernel's fp32 quantisation), and the mean error stays within the
-  bf16 bar of 5e-3.
+* The forward is judged against fp64 attention on the dequantised operands (the oracle's codes,
+  decided as above, times their scales, in fp64), within a bound per output element derived
+  from the kernel's arithmetic. The kernel rounds each probability, held as P = p * sv / sigma
+  (sigma the head's largest V scale, P <= 2^8 under the lazy max), to the nearest e4m3 value:
+  the error is at most 2^-4 * P in e4m3's normal range and at most 2^-10 (half the subnormal
+  step) below it. Summed through P V and the normalisation (the kernel's row sum, taken against
+  a running max no larger than the true one, is at least the exact l = 1 / max_j p_ij):
+    |O - O_ref| <= 2^-4 * sum_j p_ij |v_j| + 2^-10 * sigma * max_j p_ij * sum_j |code_j|
+                   + 2^-8 |O_ref| (O rounded to bf16) + 1e-3 (fp32 accumulation),
+  with the sums over the allowed keys j of row i, code_j the e4m3 value of v_j (v_j / sv_j).
+  On Gaussian inputs the mean error must also stay within the bf16 bar of 5e-3; on strongly
+  peaked rows the e4m3 floor on the many small probabilities lifts it above that (a numpy model
+  of the kernel's arithmetic gives 7.7e-3 on the peaked case below), so there the per-element
+  bound alone is the criterion.
 """
 import numpy as np
 import pytest
@@ -73,20 +80,28 @@ def test_quantize_bytes_equal_torch_float8_on_the_grid():
     np.testing.assert_array_equal(ops.q8[0, 0, 64:128].cpu().numpy(), ref)
 
 
-def _dequantised(x):
-    """The oracle's operand: fp64 quantise / dequantise of the bf16 values of one (b, h)."""
-    c, s = OF8.quantize(f64(x))
-    return OF8.dequantize(c, s)
+def _operands(x):
+    """The oracle's operand of one (b, h): codes decided in fp32 as the kernel does, their scales,
+    and the dequantised values in fp64."""
+    c, s = OF8.quantize_fp32(f64(x).astype(np.float32))
+    return c, s, OF8.dequantize(c, s)
 
 
-def _check_rows(got, q, k, v, mode, fn, rows, bias_fn=None, what=""):
-    qd, kd, vd = (_dequantised(t) for t in (q, k, v))
+def _check_rows(got, q, k, v, mode, fn, rows, bias_fn=None, what="", mean_bar=5e-3):
+    (_, _, qd), (_, _, kd), (cv, sv, vd) = (_operands(t) for t in (q, k, v))
     exp = OA.head_forward(qd, kd, vd, mode, fn, 128 ** -0.5, rows=rows, bias_fn=bias_fn)
-    bound = OA.head_forward(qd, kd, np.abs(vd), mode, fn, 128 ** -0.5, rows=rows, bias_fn=bias_fn)
+    allowed = fn(rows)
+    bias = None if bias_fn is None else bias_fn(rows)
+    p = OA.attention_probs_rows(qd[rows], kd, allowed, 128 ** -0.5, bias)
+    sigma = float(np.max(sv))
+    floor = 2.0 ** -10 * sigma * p.max(axis=1, keepdims=True) * (allowed.astype(np.float64) @ np.abs(cv))
+    bound = 2.0 ** -4 * (p @ np.abs(vd)) + floor + 2.0 ** -8 * np.abs(exp) + 1e-3
     err = np.abs(got - exp)
-    ok = err <= 2.0 ** -4 * bound + 2.0 ** -8 * np.abs(exp) + 1e-3
-    assert ok.all(), f"{what}: worst {float(err.max()):.3e} at {np.unravel_index(np.argmax(err - bound), err.shape)}"
-    assert err.mean() <= 5e-3, f"{what}: mean {float(err.mean()):.3e}"
+    ok = err <= bound
+    worst = np.unravel_index(np.argmax(err / bound), err.shape)
+    assert ok.all(), f"{what}: err {float(err[worst]):.3e} against bound {float(bound[worst]):.3e} at {worst}"
+    if mean_bar is not None:
+        assert err.mean() <= mean_bar, f"{what}: mean {float(err.mean()):.3e}"
 
 
 @pytest.mark.parametrize("N", [128 * 6, 128 * 6 + 40])
@@ -133,7 +148,7 @@ def test_forward_fp8_block_bias_and_peaked_rows():
     for h in range(H):
         bfn = OA.block_bias_fn(bias[h].numpy(), bs, bs, N)
         _check_rows(f64(o[0, h]), q[0, h], k[0, h], v[0, h], OM.HEAD_FULL, lambda r: np.ones((len(r), N), bool),
-                    np.arange(N), bias_fn=bfn, what=f"h{h}")
+                    np.arange(N), bias_fn=bfn, what=f"h{h}", mean_bar=None)
 
 
 @pytest.mark.parametrize("stride", [(1, 1, 1), (2, 4, 4)])
