@@ -870,9 +870,8 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       if (!((tile_need(sched, nseg, t, act) >> w) & 1)) continue;
-      ok = warp_all(mbar_wait(&s_full[w], (uint32_t)j & 1u, abort_flag, p.wait_limit_ns));
-      if (!ok) break;
-      tc_fence_after();
+      // The tile's schedule entries, block bias and masks depend on the
+      // schedule alone: they are worked out while its QK^T is in flight.
       const int ea = sched[2 * t];
       const int eb = (2 * t + 1 < nseg) ? sched[2 * t + 1] : -1;
       const int sa = ea & kSegIdxMask;
@@ -900,6 +899,9 @@ __global__ void __launch_bounds__(384, 1)
             mb &= geo_fast ? gna_segment_bits_geo(p.g, sb, geo[2 * t + 1], qb) : gna_segment_bits(p.g, sb, qw);
         }
       }
+      ok = warp_all(mbar_wait(&s_full[w], (uint32_t)j & 1u, abort_flag, p.wait_limit_ns));
+      if (!ok) break;
+      tc_fence_after();
       // The whole 128-key row of S is read once into registers: with its own
       // P columns, S is free for the next QK^T as soon as it has landed.
       float sv[128];

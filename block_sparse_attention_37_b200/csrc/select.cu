@@ -172,6 +172,124 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
   if (tid == 0) p.cnt[row] = base;
 }
 
+// The same selection with one warp per (b, h, query block) row and eight rows
+// per CTA (lists of at most kRowsMaxKB key blocks). The eight rows of a CTA
+// are consecutive query blocks of one (b, h), so the pooled key rows they all
+// read stay in L1; scores are made 32 keys at a time, each lane accumulating
+// its slice of the 32 dot products, and one transpose-reduction (31 shuffles)
+// leaves the full dot product of key J0 + i in lane i. Rank-and-cut and the
+// ascending compaction are warp-level (no CTA-wide barriers).
+constexpr int kRowsPerCta = 8;
+constexpr int kRowsMaxKB = 1024;
+
+// After it, lane i holds the sum over the warp of v[i] (v has 32 entries per
+// lane): five halving exchange steps, each sending half of the live values.
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      // keep v[i + (upper ? half : 0)], send the other one to the partner lane
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) select_rows_kernel(SelectParams p) {
+  extern __shared__ float rsc[];  // [kRowsPerCta][nKB] scores, then [kRowsPerCta][nKB] keep bytes
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int per_bh = (p.nQB + kRowsPerCta - 1) / kRowsPerCta;
+  const int bh = blockIdx.x / per_bh;
+  const int I = (blockIdx.x % per_bh) * kRowsPerCta + warp;
+  if (I >= p.nQB) return;  // warp-uniform; no CTA-wide barrier follows
+  const size_t row = (size_t)bh * p.nQB + I;
+  float* sc = rsc + warp * p.nKB;
+  uint8_t* keep = reinterpret_cast<uint8_t*>(rsc + kRowsPerCta * p.nKB) + warp * p.nKB;
+
+  if (p.method == BSA_SELECT_POOLED_QK) {
+    constexpr int PL = D / 32;  // channels per lane
+    float qr[PL];
+#pragma unroll
+    for (int i = 0; i < PL; ++i) qr[i] = p.qbar[row * D + lane * PL + i];
+    const float* kb = p.kbar + (size_t)bh * p.nKB * D;
+    for (int J0 = 0; J0 < p.nKB; J0 += 32) {
+      float acc[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int J = J0 + i < p.nKB ? J0 + i : p.nKB - 1;
+        const float* kr = kb + (size_t)J * D + lane * PL;
+        float a = 0.f;
+        if constexpr (PL == 4) {
+          const float4 k4 = __ldg(reinterpret_cast<const float4*>(kr));
+          a = fmaf(qr[0], k4.x, fmaf(qr[1], k4.y, fmaf(qr[2], k4.z, qr[3] * k4.w)));
+        } else {
+          const float2 k2 = __ldg(reinterpret_cast<const float2*>(kr));
+          a = fmaf(qr[0], k2.x, qr[1] * k2.y);
+        }
+        acc[i] = a;
+      }
+      const float s = transpose_reduce32(acc, lane);
+      if (J0 + lane < p.nKB) sc[J0 + lane] = sanitize(s);
+    }
+  } else {
+    const int nq = min(p.block_q, p.N - I * p.block_q);
+    for (int J = lane; J < p.nKB; J += 32) {
+      const int nk = min(p.block_k, p.N - J * p.block_k);
+      sc[J] = sanitize(p.apool[row * p.nKB + J] / ((float)nq * (float)nk));
+    }
+  }
+  for (int J = lane; J < p.nKB; J += 32) keep[J] = 0;
+  __syncwarp();
+
+  const bool full_row = p.keep_text && I < p.ntbq;
+  if (full_row) {
+    for (int J = lane; J < p.nKB; J += 32) keep[J] = 1;
+  } else {
+    if (p.keep_text)
+      for (int J = lane; J < min(p.ntbk, p.nKB); J += 32) keep[J] = 1;
+    for (int g = 0; g < p.n_groups; ++g) {
+      const int b = p.groups[g].begin, e = min(p.groups[g].end, p.nKB), k = p.groups[g].k;
+      for (int J = b + lane; J < e; J += 32) {
+        const float sj = sc[J];
+        int rank = 0;
+        for (int J2 = b; J2 < e; ++J2) {
+          const float s2 = sc[J2];
+          rank += (s2 > sj) || (s2 == sj && J2 < J);
+        }
+        if (rank < k) keep[J] = 1;
+      }
+    }
+  }
+  __syncwarp();
+
+  // ascending compaction, 32 key blocks at a time
+  int32_t* idx = p.idx + row * p.max_k;
+  uint8_t* flag = p.flag + row * p.max_k;
+  int base = 0;
+  for (int J0 = 0; J0 < p.nKB; J0 += 32) {
+    const int J = J0 + lane;
+    const bool kk = J < p.nKB && keep[J];
+    const unsigned bal = __ballot_sync(0xffffffffu, kk);
+    if (kk) {
+      const int pos = base + __popc(bal & ((1u << lane) - 1u));
+      idx[pos] = J;
+      flag[pos] = BSA_BLOCK_FULL;
+    }
+    if (J < p.nKB && p.bitmap) p.bitmap[row * p.nKB + J] = kk ? BSA_BLOCK_FULL : BSA_BLOCK_NONE;
+    base += __popc(bal);
+  }
+  for (int e = base + lane; e < p.max_k; e += 32) {
+    idx[e] = -1;
+    flag[e] = 0;
+  }
+  if (lane == 0) p.cnt[row] = base;
+}
+
 cudaError_t launch_block_pool(int d, const PoolParams& p, cudaStream_t stream) {
   dim3 grid(max(p.nQB, p.nKB), p.B * p.H, 2);
   if (d == 64)
@@ -182,6 +300,15 @@ cudaError_t launch_block_pool(int d, const PoolParams& p, cudaStream_t stream) {
 }
 
 cudaError_t launch_select(int d, const SelectParams& p, cudaStream_t stream) {
+  if (p.nKB <= kRowsMaxKB) {
+    const size_t smem = (size_t)kRowsPerCta * p.nKB * (sizeof(float) + 1);
+    const unsigned grid = (unsigned)((size_t)p.B * p.H * ((p.nQB + kRowsPerCta - 1) / kRowsPerCta));
+    if (d == 64)
+      select_rows_kernel<64><<<grid, 32 * kRowsPerCta, smem, stream>>>(p);
+    else
+      select_rows_kernel<128><<<grid, 32 * kRowsPerCta, smem, stream>>>(p);
+    return cudaGetLastError();
+  }
   const size_t smem = (size_t)p.nKB * sizeof(float) + (size_t)p.nKB;
   const unsigned grid = (unsigned)((size_t)p.B * p.H * p.nQB);
   if (d == 64)
