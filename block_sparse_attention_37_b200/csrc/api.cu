@@ -1,6 +1,7 @@
 // C ABI of the library (include/bsa.h): argument checks, TMA descriptors and
 // launches. No allocation, no host synchronisation except in
 // bsa_get_device_error, no CPU fallback.
+#include <algorithm>
 #include <atomic>
 #include <cstring>
 #include <mutex>
@@ -150,24 +151,87 @@ int check_list(const bsa_block_list* l, int nKB) {
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Workspace of the selection. POOLED_QK: qbar, kbar. FULL_SCORE, one-pass
+// form (chunk > 0): apool (block_q / 128 partial rows per query block), then
+// the per-tile LSE slabs of `chunk` query blocks, the selection running over
+// the query blocks that many at a time; two-pass form (chunk = 0): lse,
+// apool (one row per query block).
 struct SelectLayout {
-  size_t qbar, kbar, lse, apool, total;
+  size_t qbar, kbar, lse, apool, tlse, total;
+  long long chunk;
 };
 
-SelectLayout select_layout(const bsa_dims* dm, const bsa_select_spec* sp) {
-  SelectLayout L{0, 0, 0, 0, 0};
+// The one-pass slabs of one chunk take at most this many bytes in the
+// reported workspace size, so that the workspace stays bounded at any N.
+constexpr size_t kTlseCapBytes = size_t(1) << 30;
+// A one-pass chunk smaller than this many score CTAs (about three waves at
+// two CTAs per SM) would leave much of the GPU idle: the two-pass form then
+// runs instead.
+constexpr long long kOnePassMinCtas = 1024;
+
+struct FullScoreGeom {
+  long long units;    // query blocks, B * H * nQB
+  int m;              // 128-row query tiles per query block
+  size_t unit_bytes;  // slab bytes of one query block
+  long long min_chunk;
+};
+
+FullScoreGeom full_score_geom(const bsa_dims* dm) {
+  FullScoreGeom g;
+  const long long nQB = ceil_div(dm->N, dm->block_q);
+  g.units = (long long)dm->B * dm->H * nQB;
+  g.m = dm->block_q >= 128 ? dm->block_q / 128 : 1;
+  g.unit_bytes = (size_t)g.m * (size_t)ceil_div(dm->N, 128) * 128 * sizeof(float);
+  g.min_chunk = std::min(g.units, (kOnePassMinCtas + g.m - 1) / g.m);
+  return g;
+}
+
+SelectLayout two_pass_layout(const bsa_dims* dm) {
+  SelectLayout L{0, 0, 0, 0, 0, 0, 0};
   const size_t BH = (size_t)dm->B * dm->H;
   const size_t nQB = ceil_div(dm->N, dm->block_q), nKB = ceil_div(dm->N, dm->block_k);
+  L.apool = align256(BH * dm->N * sizeof(float));
+  L.total = L.apool + align256(BH * nQB * nKB * sizeof(float));
+  return L;
+}
+
+SelectLayout one_pass_layout(const bsa_dims* dm, long long chunk) {
+  SelectLayout L{0, 0, 0, 0, 0, 0, chunk};
+  const FullScoreGeom g = full_score_geom(dm);
+  const size_t nKB = ceil_div(dm->N, dm->block_k);
+  L.tlse = align256((size_t)g.units * g.m * nKB * sizeof(float));
+  L.total = L.tlse + (size_t)chunk * g.unit_bytes;
+  return L;
+}
+
+// The layout bsa_select_workspace_size reports: for FULL_SCORE the one-pass
+// form with every query block in one chunk, or as many as kTlseCapBytes holds.
+SelectLayout select_layout(const bsa_dims* dm, const bsa_select_spec* sp) {
   if (sp->method == BSA_SELECT_POOLED_QK) {
-    L.qbar = 0;
+    SelectLayout L{0, 0, 0, 0, 0, 0, 0};
+    const size_t BH = (size_t)dm->B * dm->H;
+    const size_t nQB = ceil_div(dm->N, dm->block_q), nKB = ceil_div(dm->N, dm->block_k);
     L.kbar = align256(BH * nQB * dm->d * sizeof(float));
     L.total = L.kbar + align256(BH * nKB * dm->d * sizeof(float));
-  } else {
-    L.lse = 0;
-    L.apool = align256(BH * dm->N * sizeof(float));
-    L.total = L.apool + align256(BH * nQB * nKB * sizeof(float));
+    return L;
   }
-  return L;
+  const FullScoreGeom g = full_score_geom(dm);
+  const long long cap = std::max(1ll, (long long)(kTlseCapBytes / g.unit_bytes));
+  return one_pass_layout(dm, std::min(g.units, std::max(cap, g.min_chunk)));
+}
+
+// The layout a workspace of `bytes` runs: for FULL_SCORE the one-pass form
+// with as many query blocks per chunk as the bytes hold, if that is at least
+// the minimum chunk, else the two-pass form. total > bytes: neither fits.
+SelectLayout layout_for_bytes(const bsa_dims* dm, const bsa_select_spec* sp, size_t bytes) {
+  if (sp->method == BSA_SELECT_POOLED_QK) return select_layout(dm, sp);
+  const FullScoreGeom g = full_score_geom(dm);
+  const size_t base = one_pass_layout(dm, 0).tlse;
+  if (bytes > base) {
+    const long long chunk = std::min(g.units, (long long)((bytes - base) / g.unit_bytes));
+    if (chunk >= g.min_chunk) return one_pass_layout(dm, chunk);
+  }
+  return two_pass_layout(dm);
 }
 
 // Every argument check of bsa_select_topk except the workspace's, in the
@@ -319,15 +383,30 @@ size_t bsa_select_workspace_size(const bsa_dims* dims, const bsa_select_spec* sp
   return select_layout(dims, spec).total;
 }
 
+// bsa_select_topk after its argument and workspace checks; also the body of
+// bsa_select_topk_static. Runs the form that `workspace_bytes` holds.
+static int select_topk_in(const bsa_dims* dims, const void* Q, const void* K, const bsa_select_spec* spec,
+                          const float* block_bias, void* workspace, size_t workspace_bytes,
+                          const bsa_block_list* out, void* stream);
+
 int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K, const bsa_select_spec* spec,
                     const float* block_bias, void* workspace, size_t workspace_bytes, const bsa_block_list* out,
                     void* stream) {
   int st = check_select_args(dims, Q, K, spec, out);
   if (st != BSA_OK) return st;
-  const int nQB = ceil_div(dims->N, dims->block_q), nKB = ceil_div(dims->N, dims->block_k);
-  const SelectLayout L = select_layout(dims, spec);
-  if (!workspace || workspace_bytes < L.total || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  if (!workspace || workspace_bytes < select_layout(dims, spec).total ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return BSA_ERR_WORKSPACE;
+  return select_topk_in(dims, Q, K, spec, block_bias, workspace, workspace_bytes, out, stream);
+}
+
+static int select_topk_in(const bsa_dims* dims, const void* Q, const void* K, const bsa_select_spec* spec,
+                          const float* block_bias, void* workspace, size_t workspace_bytes,
+                          const bsa_block_list* out, void* stream) {
+  int st = BSA_OK;
+  const int nQB = ceil_div(dims->N, dims->block_q), nKB = ceil_div(dims->N, dims->block_k);
+  const SelectLayout L = layout_for_bytes(dims, spec, workspace_bytes);
+  if (L.total > workspace_bytes) return BSA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
 
@@ -389,14 +468,29 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K, const bs
     ap.scale_log2 = spec->scale * 1.4426950408889634f;
     ap.wait_limit_ns = g_wait_limit_ns.load();
     ap.withhold_tile = -1;
-    ap.lse = reinterpret_cast<float*>(ws + L.lse);
     ap.apool = reinterpret_cast<float*>(ws + L.apool);
-    const int grid = (int)(BH * ap.nQT);
-    if ((st = cuda_status(launch_score(dims->d, KIND_LSE, mq, mk, ap, grid, s))) != BSA_OK) return st;
-    if ((st = cuda_status(cudaMemsetAsync(ap.apool, 0, (size_t)BH * nQB * nKB * sizeof(float), s))) != BSA_OK)
-      return st;
-    if ((st = cuda_status(launch_score(dims->d, KIND_POOL, mq, mk, ap, grid, s))) != BSA_OK) return st;
+    if (L.chunk > 0) {
+      // one pass per chunk of query blocks; each query tile writes its partial row of A'
+      const FullScoreGeom g = full_score_geom(dims);
+      ap.tlse = reinterpret_cast<float*>(ws + L.tlse);
+      for (long long u0 = 0; u0 < g.units; u0 += L.chunk) {
+        const long long n = std::min(L.chunk, g.units - u0);
+        ap.u0 = u0;
+        if ((st = cuda_status(launch_score(dims->d, KIND_TLSE, mq, mk, ap, (int)(n * g.m), s))) != BSA_OK)
+          return st;
+      }
+      sp.parts = g.m;
+    } else {
+      ap.lse = reinterpret_cast<float*>(ws + L.lse);
+      const int grid = (int)(BH * ap.nQT);
+      if ((st = cuda_status(launch_score(dims->d, KIND_LSE, mq, mk, ap, grid, s))) != BSA_OK) return st;
+      if ((st = cuda_status(cudaMemsetAsync(ap.apool, 0, (size_t)BH * nQB * nKB * sizeof(float), s))) != BSA_OK)
+        return st;
+      if ((st = cuda_status(launch_score(dims->d, KIND_POOL, mq, mk, ap, grid, s))) != BSA_OK) return st;
+      sp.parts = 1;
+    }
     sp.apool = ap.apool;
+    sp.nQT = ap.nQT;
   }
   return cuda_status(launch_select(dims->d, sp, s));
 }

@@ -5,7 +5,7 @@
 
 namespace bsa {
 
-enum { KIND_LSE = 1, KIND_POOL = 2 };
+enum { KIND_LSE = 1, KIND_POOL = 2, KIND_TLSE = 3 };
 
 // 64-key segments per sequence the per-CTA schedule can hold: N <= 131072.
 constexpr int kMaxSeg = 2048;
@@ -27,6 +27,11 @@ struct AttnParams {
   __nv_bfloat16* O;          // [B,H,N,d]
   float* lse;                // [B,H,N] log2-domain row LSE (LSE out, POOL in)
   float* apool;              // [B,H,nQB,nKB] block sums of softmax (POOL out)
+  // TLSE: per 128-row query tile (CTA c of the launch) a [T][128] slab of
+  // per-tile row LSEs, T = ceil(N/128); the launch covers the query blocks
+  // u0, u0 + 1, ... in (b, h, I) order, block_q / 128 CTAs per block
+  float* tlse;
+  long long u0;
   int has_gna;
   GnaDev g;
   // failure detection: the limit of every pipeline wait, and a tile whose K
@@ -48,7 +53,9 @@ cudaError_t launch_forward(int d, const CUtensorMap& q, const CUtensorMap& k, co
 cudaError_t launch_forward_fp8(const CUtensorMap& q8, const CUtensorMap& k8, const CUtensorMap& v8t,
                                const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream);
 
-// The two score passes of the full-score selection (score.cu); grid = B*H*ceil(N/128).
+// The score passes of the full-score selection (score.cu). KIND_LSE and
+// KIND_POOL: grid = B*H*ceil(N/128). KIND_TLSE: grid = (query blocks in the
+// chunk) * block_q / 128.
 cudaError_t launch_score(int d, int kind, const CUtensorMap& q, const CUtensorMap& k, const AttnParams& p,
                          int grid, cudaStream_t stream);
 

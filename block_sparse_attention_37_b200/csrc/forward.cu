@@ -24,6 +24,8 @@
 // Output leaves through shared memory and a TMA store.
 #include <utility>
 
+#include <type_traits>
+
 #include "tiles.cuh"
 
 namespace bsa {
@@ -110,8 +112,12 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 // Sorted union schedule of the CTA's four 64-row groups (warp 0). Returns count.
 // Warp-parallel throughout: the block-list rows of all groups are read in one
 // round of loads, and segments are emitted 32 at a time by ballot compaction.
+// Sparse GNA heads in a one-slice layout: a partial segment outside a group's
+// window loses that group's bit (the group needs neither its QK^T nor its
+// PV), and a segment no group needs is left out. `pairs`: segments are kept
+// or left out in aligned pairs (the e4m3 V loads take 128-key runs).
 __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0, uint32_t* vb,
-                                 uint32_t* pb, int32_t* sched, int lane) {
+                                 uint32_t* pb, int32_t* sched, int lane, bool pairs) {
   const int nwords = (p.nSeg + 31) >> 5;
   for (int w = lane; w < 5 * 64; w += 32) vb[w] = 0u;  // vb[4][64] then pb[64]
   __syncwarp();
@@ -182,14 +188,38 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
     }
   }
   __syncwarp();
+  // the groups' windows (lane g computes group g's, then every lane gets all four)
+  const bool narrow = mode != BSA_HEAD_FULL && p.has_gna && p.g.seg_one_slice;
+  GroupWin gw[4];
+  if (narrow) {
+    GroupWin mine{0, 0, 0, 0, 0, 0, false};
+    if (lane < 4 && row0 + 64 * lane < p.N) mine = gna_group_window(p.g, (row0 >> 6) + lane);
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      gw[g].t0 = __shfl_sync(0xffffffffu, mine.t0, g);
+      gw[g].t1 = __shfl_sync(0xffffffffu, mine.t1, g);
+      gw[g].y0 = __shfl_sync(0xffffffffu, mine.y0, g);
+      gw[g].y1 = __shfl_sync(0xffffffffu, mine.y1, g);
+      gw[g].x0 = __shfl_sync(0xffffffffu, mine.x0, g);
+      gw[g].x1 = __shfl_sync(0xffffffffu, mine.x1, g);
+      gw[g].ok = __shfl_sync(0xffffffffu, (int)mine.ok, g) != 0;
+    }
+  }
   // emit the kept segments in ascending order, 32 at a time
   int base = 0;
   for (int s0 = 0; s0 < p.nSeg; s0 += 32) {
     const int wd = s0 >> 5, s = s0 + lane;
     const uint32_t v0 = vb[wd], v1 = vb[64 + wd], v2 = vb[128 + wd], v3 = vb[192 + wd], pw = pb[wd];
-    const uint32_t gb = ((v0 >> lane) & 1u) | (((v1 >> lane) & 1u) << 1) | (((v2 >> lane) & 1u) << 2) |
-                        (((v3 >> lane) & 1u) << 3);
-    const bool keep = s < p.nSeg && gb != 0u;
+    uint32_t gb = ((v0 >> lane) & 1u) | (((v1 >> lane) & 1u) << 1) | (((v2 >> lane) & 1u) << 2) |
+                  (((v3 >> lane) & 1u) << 3);
+    if (narrow && s < p.nSeg && gb != 0u && ((pw >> lane) & 1u)) {
+      const uint64_t geo = gna_segment_geo(p.g, s);
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        if (((gb >> g) & 1u) && !gna_segment_meets(p.g, geo, gw[g])) gb &= ~(1u << g);
+    }
+    const uint32_t gp = __shfl_xor_sync(0xffffffffu, gb, 1);  // the aligned partner's bits
+    const bool keep = s < p.nSeg && (gb != 0u || (pairs && gp != 0u));
     const uint32_t bal = __ballot_sync(0xffffffffu, keep);
     if (keep)
       sched[base + __popc(bal & ((1u << lane) - 1u))] =
@@ -486,7 +516,7 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
   }
   if (warp == 0) {
-    const int n = build_schedule256(p, mode, bh, row0, vb, vb + 256, sched, lane);
+    const int n = build_schedule256(p, mode, bh, row0, vb, vb + 256, sched, lane, F8);
     // tiles each warpgroup needs
     const int act = 1 | ((row0 + 128 < p.N) ? 2 : 0);
     if constexpr (F8) reorder_tiles(sched, reinterpret_cast<int32_t*>(smem + C::TMP_OFF), n, act, lane);
@@ -550,11 +580,20 @@ __global__ void __launch_bounds__(384, 1)
   };
   if (warp < 4) {
     regs_release<C::REGS_CTL>();
-    if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    if (lane == 0 && T > 0) {
-      int k_issued = 0, v_issued = 0;
-      uint32_t kpar = 0u, vpar = 0u;  // phase parity per (stage, warpgroup) release barrier
+    if (warp == 0 || warp == 2) {
+    // ---------------------------------------------------------------- producers
+    // One ring each, in two warps (a wait of one does not hold up the other):
+    // warp 0 loads K tiles, warp 2 V tiles. A stage of either ring is
+    // reloaded once the warpgroups that used its previous tile have released
+    // it (QK^T for K, PV for V), so K runs ahead of the PVs instead of
+    // queueing behind V.
+    // the ring's loop, instantiated once per ring (no runtime branch on the kind)
+    auto produce = [&](auto ring) {
+      constexpr bool IS_K = decltype(ring)::value;
+      uint64_t* const full = IS_K ? k_full : v_full;
+      uint64_t* const empty = IS_K ? k_empty : v_empty;
+      int issued = 0;
+      uint32_t par = 0u;  // phase parity per (stage, warpgroup) release barrier
       for (int t = 0; t < T; ++t) {
         const int st = t % S;
         const int sa = sched[2 * t] & kSegIdxMask;
@@ -565,59 +604,54 @@ __global__ void __launch_bounds__(384, 1)
         for (int w = 0; w < 2 && released; ++w)
           if ((prev_need >> w) & 1) {
             const int b = 2 * st + w;
-            released = mbar_wait(&k_empty[b], (kpar >> b) & 1u, abort_flag, p.wait_limit_ns);
-            kpar ^= 1u << b;
+            released = mbar_wait(&empty[b], (par >> b) & 1u, abort_flag, p.wait_limit_ns);
+            par ^= 1u << b;
           }
         if (!released) {
           cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
           break;
         }
-        // a withheld tile (failure-detection test) is never loaded: its
-        // consumers' waits run out
-        if (t != p.withhold_tile) {
-          mbar_arrive_expect_tx(&k_full[st], C::TILE);
-          uint8_t* dk = sK + st * C::TILE;
-          for (int c = 0; c < C::NCH; ++c) {
-            tma_load_3d(dk + c * C::CHUNK, &tmK, &k_full[st], c * 64, sa * 64, bh);
-            tma_load_3d(dk + c * C::CHUNK + C::CHUNK / 2, &tmK, &k_full[st], c * 64, sb * 64, bh);
+        if constexpr (IS_K) {
+          // a withheld tile (failure-detection test) is never loaded: its
+          // consumers' waits run out
+          if (t != p.withhold_tile) {
+            mbar_arrive_expect_tx(&k_full[st], C::TILE);
+            uint8_t* dk = sK + st * C::TILE;
+            for (int c = 0; c < C::NCH; ++c) {
+              tma_load_3d(dk + c * C::CHUNK, &tmK, &k_full[st], c * 64, sa * 64, bh);
+              tma_load_3d(dk + c * C::CHUNK + C::CHUNK / 2, &tmK, &k_full[st], c * 64, sb * 64, bh);
+            }
           }
-        }
-        k_issued = t + 1;
-        for (int w = 0; w < 2 && released; ++w)
-          if ((prev_need >> w) & 1) {
-            const int b = 2 * st + w;
-            released = mbar_wait(&v_empty[b], (vpar >> b) & 1u, abort_flag, p.wait_limit_ns);
-            vpar ^= 1u << b;
-          }
-        if (!released) {
-          cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
-          break;
-        }
-        mbar_arrive_expect_tx(&v_full[st], C::TILE);
-        uint8_t* dv = sV + st * C::TILE;
-        if constexpr (F8) {
-          // V transposed: the tile's 128 keys are one 128-byte run per channel
-          // row. Key blocks of 128 or more make every tile an aligned pair of
-          // segments (the host checks); anything else is recorded, and the
-          // load still goes out so the pipeline stays whole
-          if ((sa & 1) || (2 * t + 1 < nseg && sb != sa + 1)) record_error(BSA_DEVERR_SCHEDULE);
-          for (int h2 = 0; h2 < 2; ++h2) tma_load_3d(dv + h2 * (C::CHUNK / 2), &tmV, &v_full[st], sa * 64, 64 * h2, bh);
         } else {
-          for (int c = 0; c < D / 64; ++c) {
-            tma_load_3d(dv + c * C::CHUNK, &tmV, &v_full[st], c * 64, sa * 64, bh);
-            tma_load_3d(dv + c * C::CHUNK + C::CHUNK / 2, &tmV, &v_full[st], c * 64, sb * 64, bh);
+          mbar_arrive_expect_tx(&v_full[st], C::TILE);
+          uint8_t* dv = sV + st * C::TILE;
+          if constexpr (F8) {
+            // V transposed: the tile's 128 keys are one 128-byte run per channel
+            // row. Key blocks of 128 or more make every tile an aligned pair of
+            // segments (the host checks); anything else is recorded, and the
+            // load still goes out so the pipeline stays whole
+            if ((sa & 1) || (2 * t + 1 < nseg && sb != sa + 1)) record_error(BSA_DEVERR_SCHEDULE);
+            for (int h2 = 0; h2 < 2; ++h2) tma_load_3d(dv + h2 * (C::CHUNK / 2), &tmV, &v_full[st], sa * 64, 64 * h2, bh);
+          } else {
+            for (int c = 0; c < D / 64; ++c) {
+              tma_load_3d(dv + c * C::CHUNK, &tmV, &v_full[st], c * 64, sa * 64, bh);
+              tma_load_3d(dv + c * C::CHUNK + C::CHUNK / 2, &tmV, &v_full[st], c * 64, sb * 64, bh);
+            }
           }
         }
-        v_issued = t + 1;
+        issued = t + 1;
       }
-      if (*abort_flag) {  // copies in flight land before the CTA ends
-        for (int t = k_issued - S < 0 ? 0 : k_issued - S; t < k_issued; ++t)
-          if (t != p.withhold_tile) mbar_drain(&k_full[t % S], (uint32_t)(t / S) & 1u);
-        for (int t = v_issued - S < 0 ? 0 : v_issued - S; t < v_issued; ++t)
-          mbar_drain(&v_full[t % S], (uint32_t)(t / S) & 1u);
-      }
+      if (*abort_flag)  // copies in flight land before the CTA ends
+        for (int t = issued - S < 0 ? 0 : issued - S; t < issued; ++t)
+          if (!IS_K || t != p.withhold_tile) mbar_drain(&full[t % S], (uint32_t)(t / S) & 1u);
+    };
+    if (lane == 0 && T > 0) {
+      if (warp == 0)
+        produce(std::true_type{});
+      else
+        produce(std::false_type{});
     }
-    if (lane == 0)  // every CTA loaded Q: it must have landed before the CTA ends
+    if (warp == 0 && lane == 0)  // every CTA loaded Q: it must have landed before the CTA ends
       for (int w = 0; w < 2; ++w) mbar_drain(&q_full[w], 0u);
     } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -783,8 +817,14 @@ __global__ void __launch_bounds__(384, 1)
             q = true;
           }
           // P is written over S: the previous PV must be issued first (the
-          // tensor pipe keeps issue order)
-          if ((w ? pt1 : pt0) >= 0 && !pv(w)) return false;
+          // tensor pipe keeps issue order). V of that tile reuses the stage of
+          // tile u - S, so the other warpgroup's PV of a tile <= u - S, which
+          // releases it, goes before it.
+          const int u = w ? pt1 : pt0, uo = w ? pt0 : pt1;
+          if (u >= 0) {
+            if (uo >= 0 && uo <= u - S && !pv(1 - w)) return false;
+            if (!pv(w)) return false;
+          }
           tc_fence_after();
           if constexpr (F8)
             qk8_all(tmem + C::S_COL + w * 128, smem_desc_sw128(sQa + w * C::QSLOT, 16, 1024),
@@ -807,9 +847,8 @@ __global__ void __launch_bounds__(384, 1)
         };
         bool ok = true;
         for (int t = 0; t < T && ok; ++t) {
-          // K(t) arrives only after the producer has reloaded V for tile t - 1,
-          // which needs every PV of tile t - 1 - S: issue those first
-          ok = flush_below(t - S) && wwait(&k_full[t % S], (uint32_t)(t / S) & 1u);
+          // K(t) needs only the QK^Ts of tile t - S, issued earlier in this loop
+          ok = wwait(&k_full[t % S], (uint32_t)(t / S) & 1u);
           if (!ok) break;
           const int nw = tile_need(sched, nseg, t, act);
           if (nw & 1) ok = qk(0, t);

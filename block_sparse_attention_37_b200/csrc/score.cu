@@ -1,11 +1,21 @@
-// The two score passes of the SparseD full-score selection ("Isolated
+// The score passes of the SparseD full-score selection ("Isolated
 // Selection": A = attention map, A' = avgpool(A, block_size), top-rho% per
 // query block and key group), on tcgen05 tensor cores.
 //
-//   KIND_LSE   per-row log-sum-exp (log2 units) of scale*q.k + bias over all keys
-//   KIND_POOL  given the LSE, the block sums of softmax(z), i.e. the numerators
-//              of A'[I, J]; every 128-row query tile adds its 128 rows into
-//              A'[I, J] (one atomic per warp and 64-key half)
+//   KIND_TLSE  one pass: per row and 128-key tile the log-sum-exp (log2
+//              units) of z = scale*q.k + bias over the tile's keys, kept in a
+//              [T][128] slab per query tile, and the row's LSE over all keys
+//              carried along; at the end each row reads its slab back (it is
+//              still in L2) and the CTA writes its query tile's partial row of
+//              A': sum over its rows of 2^(tile LSE - row LSE), per key block
+//   KIND_LSE   two-pass form, first pass: per-row LSE over all keys
+//   KIND_POOL  two-pass form, second pass: given the LSE, the block sums of
+//              softmax(z), i.e. the numerators of A'[I, J]; every 128-row
+//              query tile adds its 128 rows into A'[I, J] (one atomic per
+//              warp and 64-key half)
+// The one-pass form evaluates QK^T and the exps once instead of twice, and
+// its sums have a fixed order; the two-pass form needs no per-tile slabs and
+// runs where the workspace cannot hold them.
 //
 // One CTA computes one 128-row query tile of one (b, h) against every key.
 // Roles (192 threads): warp 0 TMA producer (Q once, K tiles into a ring),
@@ -46,8 +56,17 @@ __global__ void __launch_bounds__(192, 2)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qt = blockIdx.x % p.nQT;
-  const int bh = blockIdx.x / p.nQT;
+  int qt, bh;
+  if (KIND == KIND_TLSE) {
+    const int m = p.block_q >> 7;  // query tiles per query block
+    const long long u = p.u0 + blockIdx.x / m;
+    bh = (int)(u / p.nQB);
+    qt = (int)(u % p.nQB) * m + (int)(blockIdx.x % m);
+    if (qt >= p.nQT) return;  // the ragged last block of a head has fewer tiles (whole CTA, before any setup)
+  } else {
+    qt = blockIdx.x % p.nQT;
+    bh = blockIdx.x / p.nQT;
+  }
   const int h = bh % p.H;
   const int row0 = qt * 128;
   const int T = (p.N + 127) >> 7;  // 128-key tiles
@@ -155,6 +174,7 @@ __global__ void __launch_bounds__(192, 2)
     const int Iq = (row_valid ? pq : (p.N - 1)) / p.block_q;
     const size_t bias_row = ((size_t)h * p.nQB + Iq) * p.nKB;
     float m = kNegInf, l = 0.f;
+    float* tslab = KIND == KIND_TLSE ? p.tlse + (size_t)blockIdx.x * T * 128 : nullptr;
     const float lse2 = (KIND == KIND_POOL && row_valid) ? p.lse[(size_t)bh * p.N + pq] : 0.f;
     bool ok = true;
     float s[128];
@@ -177,7 +197,7 @@ __global__ void __launch_bounds__(192, 2)
       // The per-row reductions below run as several independent chains (a
       // single 128-long chain of dependent max or add instructions would
       // take longer than the exps themselves).
-      if (KIND == KIND_LSE) {
+      if (KIND != KIND_POOL) {
         // z = scale * s + bias, per 64-key half
 #pragma unroll
         for (int j = 0; j < 64; j += 2) fma2(s[j], s[j + 1], p.scale_log2, ba);
@@ -229,6 +249,39 @@ __global__ void __launch_bounds__(192, 2)
           add2(a2, a3, fast_exp2(x2), fast_exp2(x3));
         }
         l += (a0 + a1) + (a2 + a3);
+      } else if (KIND == KIND_TLSE) {
+        // the tile's own LSE: max, then the sum of exp2(z - max), no running state
+        float m0 = s[0], m1 = s[1], m2 = s[2], m3 = s[3];
+#pragma unroll
+        for (int j = 4; j < 124; j += 8) {
+          m0 = max3f(m0, s[j], s[j + 1]);
+          m1 = max3f(m1, s[j + 2], s[j + 3]);
+          m2 = max3f(m2, s[j + 4], s[j + 5]);
+          m3 = max3f(m3, s[j + 6], s[j + 7]);
+        }
+        m0 = max3f(m0, s[124], s[125]);
+        m1 = max3f(m1, s[126], s[127]);
+        const float mx = fmaxf(fmaxf(m0, m1), fmaxf(m2, m3));
+        const float mu = (mx == kNegInf) ? 0.f : mx;
+        float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 128; j += 4) {
+          float x0 = s[j], x1 = s[j + 1], x2 = s[j + 2], x3 = s[j + 3];
+          fma2(x0, x1, 1.f, -mu);
+          fma2(x2, x3, 1.f, -mu);
+          add2(a0, a1, fast_exp2(x0), fast_exp2(x1));
+          add2(a2, a3, fast_exp2(x2), fast_exp2(x3));
+        }
+        const float lt = (a0 + a1) + (a2 + a3);
+        const float xt = (lt > 0.f) ? mx + __log2f(lt) : kNegInf;
+        // consecutive rows are consecutive floats: one 128-byte store per warp
+        if (row_valid) tslab[(size_t)t * 128 + r] = xt;
+        // the row's LSE over the tiles so far, as a running (max, sum)
+        if (xt > kNegInf) {
+          const float mn = fmaxf(m, xt);
+          l = l * fast_exp2(m - mn) + fast_exp2(xt - mn);
+          m = mn;
+        }
       } else {
         // block sums of exp2(z - lse) per 64-key half, two packed accumulators each
         float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f, b0 = 0.f, b1 = 0.f, b2 = 0.f, b3 = 0.f;
@@ -260,6 +313,47 @@ __global__ void __launch_bounds__(192, 2)
     }
     if (!ok) cta_fail(abort_flag, BSA_DEVERR_TIMEOUT);
     if (KIND == KIND_LSE && row_valid) p.lse[(size_t)bh * p.N + pq] = (l > 0.f) ? m + __log2f(l) : kNegInf;
+    if (KIND == KIND_TLSE) {
+      // The query tile's partial row of A'. Every MMA has completed (each
+      // softmax warp saw the last S land), so the K ring is free: it holds
+      // one row of per-warp sums per warp, added in a fixed order. All four
+      // warps reach the barrier; in an aborting CTA (where copies into the
+      // ring may still be in flight) none of them touches it.
+      const bool live = ok && row_valid && l > 0.f;
+      const float lse = live ? m + __log2f(l) : 0.f;
+      const int tpk = p.block_k >> 7;  // 128-key tiles per key block
+      float* red = reinterpret_cast<float*>(sK);
+      for (int J0 = 0; J0 < p.nKB; J0 += 32) {
+        float acc[32];
+        if (tpk == 1) {
+          // one tile per key block: 32 independent loads in flight, then the exps
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            acc[i] = (live && J0 + i < p.nKB) ? tslab[(size_t)(J0 + i) * 128 + r] : kNegInf;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) acc[i] = fast_exp2(acc[i] - lse);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int J = J0 + i;
+            float a = 0.f;
+            if (live && J < p.nKB) {
+              const int t1 = min((J + 1) * tpk, T);
+              for (int t = J * tpk; t < t1; ++t) a += fast_exp2(tslab[(size_t)t * 128 + r] - lse);
+            }
+            acc[i] = a;
+          }
+        }
+        const float sum = transpose_reduce32(acc, lane);
+        if (ok && J0 + lane < p.nKB) red[q4 * p.nKB + J0 + lane] = sum;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!*abort_flag) {
+        float* dst = p.apool + ((size_t)p.u0 * (p.block_q >> 7) + blockIdx.x) * p.nKB;
+        for (int J = r; J < p.nKB; J += 128)
+          dst[J] = (red[J] + red[p.nKB + J]) + (red[2 * p.nKB + J] + red[3 * p.nKB + J]);
+      }
+    }
   }
 
   tc_fence_before();
@@ -285,9 +379,12 @@ static cudaError_t launch_score_d(const CUtensorMap& q, const CUtensorMap& k, co
 
 cudaError_t launch_score(int d, int kind, const CUtensorMap& q, const CUtensorMap& k, const AttnParams& p,
                          int grid, cudaStream_t stream) {
-  if (d == 64)
+  if (d == 64) {
+    if (kind == KIND_TLSE) return launch_score_d<64, KIND_TLSE>(q, k, p, grid, stream);
     return kind == KIND_LSE ? launch_score_d<64, KIND_LSE>(q, k, p, grid, stream)
                             : launch_score_d<64, KIND_POOL>(q, k, p, grid, stream);
+  }
+  if (kind == KIND_TLSE) return launch_score_d<128, KIND_TLSE>(q, k, p, grid, stream);
   return kind == KIND_LSE ? launch_score_d<128, KIND_LSE>(q, k, p, grid, stream)
                           : launch_score_d<128, KIND_POOL>(q, k, p, grid, stream);
 }

@@ -1,21 +1,33 @@
 // Content-driven block selection.
 //  * block_pool_kernel: mean of every 64/128/256-token block of Q and K in
 //    fp32 (lmnt.cn BSA post, section 2.2, mean-pooled block vectors). HBM
-//    bound: 16-byte coalesced loads, eight blocks of loads in flight per CTA.
+//    bound: one bulk copy of the block's rows into shared memory per CTA.
 //  * select_kernel: per (b, h, query block) row, the score of every KV block
 //    (pooled dot product, or the SparseD avg-pooled softmax mass from the
-//    attention kernel's POOL pass), then an exact rank-and-cut per key group
-//    (descending score, ties to the lower index) and an ascending block list.
+//    block sums of A' the score kernel writes), then an exact cut per key
+//    group (descending score, ties to the lower index) and an ascending
+//    block list.
 #include "select.cuh"
+#include "tiles.cuh"
 
 namespace bsa {
 
 // grid: (nB, B*H, 2 tensors); block 256. out[t][bh][I][:] = mean of block I.
+// The block's rows are one contiguous run of rows * D * 2 bytes: one thread
+// moves it into shared memory with bulk copies of up to kPoolChunkRows rows
+// (no registers hold data in flight, so many CTAs per SM keep HBM busy),
+// then every thread adds its 16-byte column chunk over rows rr, rr + RPI, ...
+// in order, and the RPI partial rows are added in order.
+constexpr int kPoolChunkRows = 256;
+
 template <int D>
 __global__ void __launch_bounds__(256) block_pool_kernel(PoolParams p) {
   constexpr int CH = D / 8;           // 16-byte chunks per row
-  constexpr int RPI = 256 / CH;       // rows per iteration
+  constexpr int RPI = 256 / CH;       // rows per step
+  extern __shared__ __align__(128) uint8_t rows_smem[];  // [rows][D] bf16
   __shared__ float red[RPI][D + 1];
+  __shared__ __align__(8) uint64_t full;
+  __shared__ int no_abort;
   const int I = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int bs = which ? p.block_k : p.block_q;
   const int nb = which ? p.nKB : p.nQB;
@@ -24,23 +36,39 @@ __global__ void __launch_bounds__(256) block_pool_kernel(PoolParams p) {
   float* dst = (which ? p.kbar : p.qbar) + ((size_t)bh * nb + I) * D;
   const int r0 = I * bs;
   const int rows = min(bs, p.N - r0);
+  if (threadIdx.x == 0) {
+    no_abort = 0;
+    mbar_init(&full, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
   const int c = threadIdx.x % CH, rr = threadIdx.x / CH;
+  const uint4* rowp = reinterpret_cast<const uint4*>(rows_smem) + c;
   float acc[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-  for (int base = 0; base < rows; base += RPI * 4) {
-    uint4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int r = base + u * RPI + rr;
-      if (r < rows)
-        v[u] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)(r0 + r) * D) + c);
-      else
-        v[u] = make_uint4(0u, 0u, 0u, 0u);
+  uint32_t phase = 0u;
+  // chunks start at multiples of kPoolChunkRows (a multiple of RPI), so each
+  // thread still visits its rows rr, rr + RPI, ... in order
+  for (int c0 = 0; c0 < rows; c0 += kPoolChunkRows) {
+    const int n = min(kPoolChunkRows, rows - c0);
+    if (threadIdx.x == 0) {
+      fence_proxy_async_smem();  // the previous chunk's reads come before the copy over them
+      mbar_arrive_expect_tx(&full, (uint32_t)n * D * 2);
+      bulk_load_1d(rows_smem, src + (size_t)(r0 + c0) * D, (uint32_t)n * D * 2, &full);
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+    if (!mbar_wait(&full, phase, &no_abort)) {
+      // the copy never landed: wait (bounded) so nothing is in flight at exit
+      if (threadIdx.x == 0) {
+        record_error(BSA_DEVERR_TIMEOUT);
+        mbar_drain(&full, phase);
+      }
+      return;
+    }
+    phase ^= 1u;
+    for (int r = rr; r < n; r += RPI) {
+      const uint4 v = rowp[(size_t)r * CH];
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f = __bfloat1622float2(h2[j]);
@@ -48,6 +76,7 @@ __global__ void __launch_bounds__(256) block_pool_kernel(PoolParams p) {
         acc[2 * j + 1] += f.y;
       }
     }
+    __syncthreads();  // every thread is done with the chunk before the next copy
   }
 #pragma unroll
   for (int j = 0; j < 8; ++j) red[rr][c * 8 + j] = acc[j];
@@ -61,6 +90,14 @@ __global__ void __launch_bounds__(256) block_pool_kernel(PoolParams p) {
 }
 
 __device__ __forceinline__ float sanitize(float x) { return (x == x) ? x : -__int_as_float(0x7f800000); }
+
+// An unsigned key whose order is the float order of a non-NaN score; -0 and
+// +0 (equal as floats) map to one key.
+__device__ __forceinline__ uint32_t order_key(float x) {
+  uint32_t u = __float_as_uint(x);
+  if (u == 0x80000000u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
 
 // One CTA per (b, h, query block). Block 256 threads.
 template <int D>
@@ -112,9 +149,12 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
     }
   } else {
     const int nq = min(p.block_q, p.N - I * p.block_q);
+    const int np = min(p.parts, p.nQT - I * p.parts);  // partial rows that exist
     for (int J = tid; J < p.nKB; J += 256) {
       const int nk = min(p.block_k, p.N - J * p.block_k);
-      sc[J] = sanitize(p.apool[row * p.nKB + J] / ((float)nq * (float)nk));
+      float a = 0.f;
+      for (int j = 0; j < np; ++j) a += p.apool[((size_t)row * p.parts + j) * p.nKB + J];
+      sc[J] = sanitize(a / ((float)nq * (float)nk));
     }
   }
   for (int J = tid; J < p.nKB; J += 256) keep[J] = 0;
@@ -177,26 +217,54 @@ __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
 // are consecutive query blocks of one (b, h), so the pooled key rows they all
 // read stay in L1; scores are made 32 keys at a time, each lane accumulating
 // its slice of the 32 dot products, and one transpose-reduction (31 shuffles)
-// leaves the full dot product of key J0 + i in lane i. Rank-and-cut and the
-// ascending compaction are warp-level (no CTA-wide barriers).
+// leaves the full dot product of key J0 + i in lane i. The cut of each group
+// is a warp-wide radix select of its k-th largest score (32 counting steps,
+// linear in the group's size); it and the ascending compaction are
+// warp-level (no CTA-wide barriers).
 constexpr int kRowsPerCta = 8;
 constexpr int kRowsMaxKB = 1024;
 
-// After it, lane i holds the sum over the warp of v[i] (v has 32 entries per
-// lane): five halving exchange steps, each sending half of the live values.
-__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+
+// Keep the k largest scores of sc[b, e) (0 < k < e - b <= 32 * NPL), ties to
+// the lower index, by a warp-wide radix select of the k-th largest order key,
+// one bit at a time from the top. After the loop `prefix` is that key and
+// `kr` its rank among the keys equal to it: keys above it are kept, and of
+// the keys equal to it the kr with the lowest block indices - the same k
+// blocks as ranking by descending score with ties to the lower index. Each
+// lane holds the keys of b + lane + 32q in registers; padding keys are 0,
+// below every score's key (order_key(-inf) = 0x007fffff).
+template <int NPL>
+__device__ __forceinline__ void radix_cut(const float* sc, uint8_t* keep, int b, int e, int k, int lane) {
+  uint32_t key[NPL];
 #pragma unroll
-  for (int half = 16; half >= 1; half >>= 1) {
-    const bool upper = (lane & half) != 0;
-#pragma unroll
-    for (int i = 0; i < half; ++i) {
-      // keep v[i + (upper ? half : 0)], send the other one to the partner lane
-      const float send = upper ? v[i] : v[i + half];
-      const float keep = upper ? v[i + half] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
-    }
+  for (int q = 0; q < NPL; ++q) {
+    const int J = b + lane + 32 * q;
+    key[q] = J < e ? order_key(sc[J]) : 0u;
   }
-  return v[0];
+  uint32_t prefix = 0u, pmask = 0u;
+  int kr = k;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t bm = 1u << bit, want = prefix | bm, m = pmask | bm;
+    int c = 0;
+#pragma unroll
+    for (int q = 0; q < NPL; ++q) c += (key[q] & m) == want;
+    c = __reduce_add_sync(0xffffffffu, c);
+    if (c >= kr)
+      prefix = want;
+    else
+      kr -= c;
+    pmask = m;
+  }
+  int taken = 0;
+#pragma unroll
+  for (int q = 0; q < NPL; ++q) {
+    const int J = b + lane + 32 * q;
+    const bool eq = key[q] == prefix;  // padding keys are never equal (prefix >= 0x007fffff)
+    const unsigned be = __ballot_sync(0xffffffffu, eq);
+    if (key[q] > prefix || (eq && taken + __popc(be & ((1u << lane) - 1u)) < kr)) keep[J] = 1;
+    taken += __popc(be);
+  }
 }
 
 template <int D>
@@ -238,9 +306,12 @@ __global__ void __launch_bounds__(256) select_rows_kernel(SelectParams p) {
     }
   } else {
     const int nq = min(p.block_q, p.N - I * p.block_q);
+    const int np = min(p.parts, p.nQT - I * p.parts);  // partial rows that exist
     for (int J = lane; J < p.nKB; J += 32) {
       const int nk = min(p.block_k, p.N - J * p.block_k);
-      sc[J] = sanitize(p.apool[row * p.nKB + J] / ((float)nq * (float)nk));
+      float a = 0.f;
+      for (int j = 0; j < np; ++j) a += p.apool[((size_t)row * p.parts + j) * p.nKB + J];
+      sc[J] = sanitize(a / ((float)nq * (float)nk));
     }
   }
   for (int J = lane; J < p.nKB; J += 32) keep[J] = 0;
@@ -254,15 +325,24 @@ __global__ void __launch_bounds__(256) select_rows_kernel(SelectParams p) {
       for (int J = lane; J < min(p.ntbk, p.nKB); J += 32) keep[J] = 1;
     for (int g = 0; g < p.n_groups; ++g) {
       const int b = p.groups[g].begin, e = min(p.groups[g].end, p.nKB), k = p.groups[g].k;
-      for (int J = b + lane; J < e; J += 32) {
-        const float sj = sc[J];
-        int rank = 0;
-        for (int J2 = b; J2 < e; ++J2) {
-          const float s2 = sc[J2];
-          rank += (s2 > sj) || (s2 == sj && J2 < J);
-        }
-        if (rank < k) keep[J] = 1;
+      if (k >= e - b) {
+        for (int J = b + lane; J < e; J += 32) keep[J] = 1;
+        continue;
       }
+      if (k <= 0) continue;
+      const int per = (e - b + 31) >> 5;  // keys per lane
+      if (per <= 1)
+        radix_cut<1>(sc, keep, b, e, k, lane);
+      else if (per <= 2)
+        radix_cut<2>(sc, keep, b, e, k, lane);
+      else if (per <= 4)
+        radix_cut<4>(sc, keep, b, e, k, lane);
+      else if (per <= 8)
+        radix_cut<8>(sc, keep, b, e, k, lane);
+      else if (per <= 16)
+        radix_cut<16>(sc, keep, b, e, k, lane);
+      else
+        radix_cut<32>(sc, keep, b, e, k, lane);
     }
   }
   __syncwarp();
@@ -290,13 +370,23 @@ __global__ void __launch_bounds__(256) select_rows_kernel(SelectParams p) {
   if (lane == 0) p.cnt[row] = base;
 }
 
-cudaError_t launch_block_pool(int d, const PoolParams& p, cudaStream_t stream) {
+template <int D>
+static cudaError_t launch_block_pool_d(const PoolParams& p, cudaStream_t stream) {
+  // dynamic shared memory: one chunk of the larger block's rows (at most 64 KB)
+  static DeviceOnce once;
+  const cudaError_t e = once.run([&]() -> cudaError_t {
+    return cudaFuncSetAttribute(block_pool_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                kPoolChunkRows * D * 2);
+  });
+  if (e != cudaSuccess) return e;
+  const int rows = min(max(p.block_q, p.block_k), kPoolChunkRows);
   dim3 grid(max(p.nQB, p.nKB), p.B * p.H, 2);
-  if (d == 64)
-    block_pool_kernel<64><<<grid, 256, 0, stream>>>(p);
-  else
-    block_pool_kernel<128><<<grid, 256, 0, stream>>>(p);
+  block_pool_kernel<D><<<grid, 256, (size_t)rows * D * 2, stream>>>(p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_block_pool(int d, const PoolParams& p, cudaStream_t stream) {
+  return d == 64 ? launch_block_pool_d<64>(p, stream) : launch_block_pool_d<128>(p, stream);
 }
 
 cudaError_t launch_select(int d, const SelectParams& p, cudaStream_t stream) {

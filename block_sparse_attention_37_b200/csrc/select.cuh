@@ -21,7 +21,11 @@ struct SelectParams {
   bsa_key_group groups[4];
   const float* qbar;
   const float* kbar;
-  const float* apool;  // [B,H,nQB,nKB] block sums of softmax (FULL_SCORE)
+  // FULL_SCORE: block sums of softmax, [B*H*nQB*parts][nKB]; the `parts`
+  // rows of a query block add up to its row of A' (one per 128-row query
+  // tile of the block; a ragged last block has fewer, its others unread)
+  const float* apool;
+  int parts, nQT;
   int32_t* cnt;
   int32_t* idx;
   uint8_t* flag;

@@ -41,9 +41,12 @@ extern "C" int bsa_select_topk_static(const bsa_dims* dims, const void* Q, const
   // for the scratch.
   const int arg = bsa::check_select_args(dims, Q, K, spec, out);
   if (arg != BSA_OK) return arg;
-  if (bsa_select_workspace_size(dims, spec) > (size_t)BSA_STATIC_SCRATCH_BYTES) return BSA_ERR_WORKSPACE;
+  // the form the scratch holds: for FULL_SCORE the one-pass form if its
+  // slabs fit, else the two-pass form
+  if (bsa::layout_for_bytes(dims, spec, BSA_STATIC_SCRATCH_BYTES).total > (size_t)BSA_STATIC_SCRATCH_BYTES)
+    return BSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   const int st = bsa::scratch_for_current_device(&scratch);
   if (st != BSA_OK) return st;
-  return bsa_select_topk(dims, Q, K, spec, block_bias, scratch, (size_t)BSA_STATIC_SCRATCH_BYTES, out, stream);
+  return select_topk_in(dims, Q, K, spec, block_bias, scratch, (size_t)BSA_STATIC_SCRATCH_BYTES, out, stream);
 }

@@ -195,6 +195,23 @@ __host__ __device__ inline uint64_t gna_segment_geo(const GnaDev& g, int seg) {
   return (uint64_t)t | ((uint64_t)y0 << 17) | ((uint64_t)x0 << 34);
 }
 
+// After it, lane i holds the sum over the warp of v[i] (v has 32 entries per
+// lane): five halving exchange steps, each sending half of the live values.
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int half = 16; half >= 1; half >>= 1) {
+    const bool upper = (lane & half) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      // keep v[i + (upper ? half : 0)], send the other one to the partner lane
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+    }
+  }
+  return v[0];
+}
+
 struct QBox {
   int tlo, thi, ylo, yhi, xlo, xhi;
 };
@@ -226,6 +243,44 @@ __host__ __device__ __forceinline__ uint64_t gna_segment_bits_geo(const GnaDev& 
   const int Tx = g.tile[2];
   const uint64_t xb = bit_range64(b.xlo - x0, b.xhi - x0) & g.x_mask;
   return (xb * g.x_rep) & bit_range64(rlo * Tx, rhi * Tx);
+}
+
+// The window of a GNA query group (64 rows that form one box of the grid in a
+// one-slice layout), as the bounding box of its rows' windows: per dimension
+// [start(first coordinate), start(last coordinate) + window). The window
+// start is nondecreasing in the coordinate, so every row's window lies
+// inside it. `ok` is false for a group of text rows or one that reaches past
+// the grid (padding rows), whose rows see every key: such a group is never
+// narrowed.
+struct GroupWin {
+  int t0, t1, y0, y1, x0, x1;
+  bool ok;
+};
+
+__host__ __device__ inline GroupWin gna_group_window(const GnaDev& g, int qseg) {
+  GroupWin w{0, 0, 0, 0, 0, 0, false};
+  const uint64_t geo = gna_segment_geo(g, qseg);
+  if (geo & kGeoText) return w;
+  const int t = (int)(geo & 0x1FFFFull), y = (int)((geo >> 17) & 0x1FFFFull), x = (int)((geo >> 34) & 0x1FFFFull);
+  const int ny = g.seg_rows, nx = g.tile[2];
+  if (t >= g.grid[0] || y + ny > g.grid[1] || x + nx > g.grid[2]) return w;
+  w.t0 = gna_window_start(t, g.grid[0], g.win[0], g.stride[0]);
+  w.t1 = w.t0 + g.win[0];
+  w.y0 = gna_window_start(y, g.grid[1], g.win[1], g.stride[1]);
+  w.y1 = gna_window_start(y + ny - 1, g.grid[1], g.win[1], g.stride[1]) + g.win[1];
+  w.x0 = gna_window_start(x, g.grid[2], g.win[2], g.stride[2]);
+  w.x1 = gna_window_start(x + nx - 1, g.grid[2], g.win[2], g.stride[2]) + g.win[2];
+  w.ok = true;
+  return w;
+}
+
+// Does a key segment (one-slice layout; `geo` from gna_segment_geo) have a key
+// inside the group window? A segment outside it is masked for every row of
+// the group: the mask is the product of one interval test per dimension.
+__host__ __device__ __forceinline__ bool gna_segment_meets(const GnaDev& g, uint64_t geo, const GroupWin& w) {
+  if (!w.ok || (geo & kGeoText)) return true;
+  const int t = (int)(geo & 0x1FFFFull), y = (int)((geo >> 17) & 0x1FFFFull), x = (int)((geo >> 34) & 0x1FFFFull);
+  return t >= w.t0 && t < w.t1 && y < w.y1 && y + g.seg_rows > w.y0 && x < w.x1 && x + g.tile[2] > w.x0;
 }
 
 }  // namespace bsa

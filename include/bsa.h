@@ -142,7 +142,12 @@ const char* bsa_error_string(int status);
 int bsa_build_mask(const bsa_dims* dims, const bsa_mask_spec* spec,
                    const bsa_block_list* out, void* stream);
 
-/* Workspace bytes bsa_select_topk needs for these dims and spec. */
+/* Workspace bytes bsa_select_topk needs for these dims and spec. POOLED_QK:
+ * the pooled Q and K blocks, fp32. FULL_SCORE: A' (B*H*nQB*nKB floats)
+ * plus the per-tile row LSEs of the one-pass form, 4 * ceil(N/128) * block_q
+ * bytes per query block, for all B*H*nQB query blocks or as many as 1 GiB
+ * holds (the selection then runs over the query blocks in chunks of that
+ * many): e.g. 1.07 GB at 32 heads x 32768 tokens, block 128. */
 size_t bsa_select_workspace_size(const bsa_dims* dims, const bsa_select_spec* spec);
 
 /* bsa_select_topk: content-driven block selection.
@@ -153,7 +158,9 @@ size_t bsa_select_workspace_size(const bsa_dims* dims, const bsa_select_spec* sp
  *    k) and text query rows keep every block.
  *  FULL_SCORE (SparseD, "Isolated Selection"): A = softmax(scale*QK^T + bias)
  *    over all keys, A' = avgpool(A, block); each group (e.g. prefill and
- *    generation key blocks) keeps its own top k per query block.
+ *    generation key blocks) keeps its own top k per query block. QK^T and
+ *    its exps are evaluated once: the log-sum-exp of every row over every
+ *    128-key tile, then each row's LSE and A' from those alone.
  *  block_bias: optional device fp32 [H, nQB, nKB] logit offset (FULL_SCORE).
  *  Writes the block list (all entries FULL). Workspace: device, at least
  *  bsa_select_workspace_size bytes, 256-byte aligned; contents are scratch.
@@ -166,7 +173,8 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K,
 
 /* Size of the library-owned scratch behind bsa_select_topk_static: 16 MiB,
  * enough for the pooled selection at 24 heads x 16896 tokens (3.2 MB) and the
- * full-score selection at 32 heads x 32768 tokens (12 MB). */
+ * full-score selection at 32 heads x 32768 tokens (12 MB in its two-pass
+ * form, below). */
 #define BSA_STATIC_SCRATCH_BYTES (16u << 20)
 
 /* bsa_select_topk_static: bsa_select_topk without a caller workspace. The
@@ -175,8 +183,14 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K,
  * buffer ahead in a fixed arena, or latency-critical loops that must not
  * call cudaMalloc (which can synchronise the device) - but still own Q, K
  * and the block list.
- *  Same arguments and results as bsa_select_topk, minus the workspace. The
- *  scratch is a fixed BSA_STATIC_SCRATCH_BYTES array inside the library; every
+ *  Same arguments and results as bsa_select_topk, minus the workspace. For
+ *  FULL_SCORE the scratch runs the one-pass form when it holds the per-tile
+ *  LSEs of at least 1024 query tiles (or of all of them), in as many chunks
+ *  as it takes; otherwise the two-pass form: a first pass over QK^T for each
+ *  row's LSE (B*H*N floats), a second that adds exp2(z - LSE) into A' (B*H*
+ *  nQB*nKB floats). The two forms round differently, so a near-tie between
+ *  two key blocks may fall the other way than in bsa_select_topk.
+ *  The scratch is a fixed BSA_STATIC_SCRATCH_BYTES array inside the library; every
  *  GPU that loads the library holds it until the process exits. Nothing is
  *  allocated: no cudaMalloc, no cudaFree, no allocating library call.
  *  The first call on a device looks up the array's device address
@@ -189,9 +203,10 @@ int bsa_select_topk(const bsa_dims* dims, const void* Q, const void* K,
  *  (the kernels clear what must start at zero). Calls whose kernels overlap on
  *  the GPU (e.g. on two streams) race on the scratch: serialise them.
  *  Errors: bsa_select_topk's argument checks run first and give the same
- *  INVALID_ARG / UNSUPPORTED status; then BSA_ERR_WORKSPACE when
- *  bsa_select_workspace_size(dims, spec) exceeds BSA_STATIC_SCRATCH_BYTES;
- *  then the CUDA errors of bsa_select_topk. */
+ *  INVALID_ARG / UNSUPPORTED status; then BSA_ERR_WORKSPACE when neither
+ *  form fits in BSA_STATIC_SCRATCH_BYTES (POOLED_QK: when
+ *  bsa_select_workspace_size exceeds it); then the CUDA errors of
+ *  bsa_select_topk. */
 int bsa_select_topk_static(const bsa_dims* dims, const void* Q, const void* K,
                            const bsa_select_spec* spec, const float* block_bias,
                            const bsa_block_list* out, void* stream);

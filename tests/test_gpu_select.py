@@ -103,6 +103,20 @@ def test_full_score_select_small(N):
     _check_full(shape, q, k, groups, bias, cls)
 
 
+@pytest.mark.parametrize("N,bs,d", [(256 * 5 + 70, 256, 64), (384 * 3 + 200, 384, 128)])
+def test_full_score_select_multi_tile_blocks(N, bs, d):
+    """Blocks of two and three 128-token tiles: a query block's rows span several score CTAs, a
+    key block several per-tile LSEs; ragged last blocks; every row against the oracle."""
+    B, H = 1, 2
+    q, k, _ = W.qkv_normal(B, H, N, d, N + 7)
+    shape = W.Shape(B, H, N, d, bs, bs, 0)
+    nb = -(-N // bs)
+    groups = [(0, nb - 1, 2), (nb - 1, nb, 1)]
+    bias, _ = W.dlm_bias(H, nb, nb - 1, seed=9, n_col_pre=1, n_col_gen=1, windows=(1,))
+    cls = _select(shape, q, k, bsa().SELECT_FULL_SCORE, groups, False, d ** -0.5, bias)
+    _check_full(shape, q, k, groups, bias, cls)
+
+
 def test_full_score_select_zero_q_takes_lowest_indices():
     B, H, N, d, bs = 1, 1, 128 * 6, 128, 128
     q = torch.zeros(B, H, N, d, dtype=torch.bfloat16)

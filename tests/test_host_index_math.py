@@ -49,6 +49,17 @@ extern "C" int h_gna_classes(int n_text, const bsa_gna_geom* geom, unsigned char
     for (int J = 0; J < nb; ++J) out[I * nb + J] = (unsigned char)bsa::gna_class(g, I, J);
   return 0;
 }
+extern "C" int h_group_meets(int n_text, const bsa_gna_geom* geom, unsigned char* out, int nseg) {
+  bsa::GnaDev g;
+  const int st = bsa::make_gna(geom, n_text, &g);
+  if (st) return st;
+  if (!g.seg_one_slice) return -1;
+  for (int q = 0; q < nseg; ++q) {
+    const bsa::GroupWin w = bsa::gna_group_window(g, q);
+    for (int s = 0; s < nseg; ++s) out[q * nseg + s] = bsa::gna_segment_meets(g, bsa::gna_segment_geo(g, s), w);
+  }
+  return 0;
+}
 extern "C" void h_fdiv_many(int d, const int* n, long long* out, int count) {
   const bsa::FastDiv f = bsa::make_fastdiv(d);
   for (int i = 0; i < count; ++i) out[i] = bsa::fdiv(n[i], f);
@@ -82,6 +93,7 @@ def host_lib(tmp_path_factory):
     lib.h_gna_classes.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.h_fdiv_many.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.h_segbits_geo_row.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int]
+    lib.h_group_meets.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return lib
 
 
@@ -168,6 +180,36 @@ def test_precomputed_geometry_bits_equal_the_token_mask(host_lib, n_text, grid, 
         got = ((out[:, None] >> shifts[None, :]) & np.uint64(1)).astype(bool).reshape(-1)[:lay.N]
         exp = OM.gna_token_mask(lay, [int(pq)])[0]
         assert np.array_equal(got, exp), (grid, int(pq), np.nonzero(got != exp)[0][:5])
+
+
+@pytest.mark.parametrize("n_text,grid,tile,window,stride", CASES)
+def test_group_window_never_drops_a_visible_key(host_lib, n_text, grid, tile, window, stride):
+    """The schedule leaves a partial key segment out of a 64-row query group when it misses the
+    group's window (bounding box of its rows' windows). Wherever it does, the token mask of those
+    64 rows and 64 keys must be all false; for the video workload the test finds every empty pair
+    of an image group (the bound is tight for a box of rows)."""
+    lay = OM.GnaLayout(n_text, grid, tile, window, stride)
+    g = _geom(grid, tile, window, stride)
+    nseg = -(-lay.N // 64)
+    meets = np.zeros((nseg, nseg), dtype=np.uint8)
+    st = host_lib.h_group_meets(n_text, ctypes.byref(g), meets.ctypes.data, nseg)
+    if st == -1:
+        pytest.skip("segments span several t-slices: the schedule is not narrowed")
+    assert st == 0
+    qs = np.arange(nseg)
+    if nseg > 96:
+        qs = np.sort(np.random.default_rng(nseg).choice(nseg, 96, replace=False))
+    missed = dropped = 0
+    for q in qs:
+        rows = np.arange(64 * q, min(64 * q + 64, lay.N))
+        tm = OM.gna_token_mask(lay, rows)
+        seen = np.array([tm[:, 64 * s:64 * s + 64].any() for s in range(nseg)])
+        assert not (seen & (meets[q] == 0)).any(), (q, np.nonzero(seen & (meets[q] == 0))[0][:5])
+        dropped += int((meets[q] == 0).sum())
+        if lay.valid(rows).all() and rows[0] >= lay.text_span:
+            missed += int((~seen & (meets[q] == 1)).sum())
+    if (n_text, grid, tile, window, stride) == CASES[5]:
+        assert dropped > 0 and missed == 0
 
 
 @pytest.mark.parametrize("n_text,grid,tile,window,stride", CASES)

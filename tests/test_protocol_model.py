@@ -16,8 +16,11 @@ random ones. Checked:
   reads, no stage is reloaded while an issued MMA still reads it, and the
   softmax never overwrites P that a pending PV reads.
 
-Two planted mistakes (the fixed order without its flushes; the polling
-issuer testing K without walking the tiles in order) must be caught.
+The producer's K and V loads run as two independent agents (one lane each).
+Three planted mistakes must be caught: the fixed order without the
+cross-warpgroup PV order the split producer needs, the fixed order without
+the flushes an earlier single-loop producer needed, and the polling issuer
+testing K without walking the tiles in order.
 """
 import random
 
@@ -45,8 +48,12 @@ class Stale(AssertionError):
     pass
 
 
-def run(need, S, sep_p, seed, plant=None, max_steps=400000):
-    """need[t]: bit w = warpgroup w needs tile t. Returns 'ok' or 'deadlock'."""
+def run(need, S, sep_p, seed, plant=None, max_steps=400000, split=True):
+    """need[t]: bit w = warpgroup w needs tile t. Returns 'ok' or 'deadlock'.
+
+    split: the producer's K and V loads run as two independent agents (one lane
+    each), as in the kernel; False models the earlier single loop that loaded
+    K(t) then V(t)."""
     rng = random.Random(seed)
     T = len(need)
     B = {}
@@ -76,26 +83,35 @@ def run(need, S, sep_p, seed, plant=None, max_steps=400000):
         yield True
 
     # ---------------------------------------------------------------- producer
+    def load(kind, t, par):
+        st = t % S
+        stage, landed = (stage_k, landed_k) if kind == 'k' else (stage_v, landed_v)
+        prev = need[t - S] if t >= S else 0
+        for w in range(2):
+            if (prev >> w) & 1:
+                b = f'{kind}_empty{st}_{w}'
+                p = par.get(b, 0)
+                yield from wait(lambda b=b, p=p: bar(b).test(p))
+                par[b] = p ^ 1
+        if any(op['reads'] == (kind, st) for op in pipe):
+            raise Stale(f'{kind} stage {st} reloaded while an MMA reads it')
+        stage[st] = t
+        landed[st] = False
+        tma(kind, st, t)
+
     def producer():
         for w in range(2):
             if any((n >> w) & 1 for n in need):
                 events.append(lambda w=w: bar(f'q_full{w}').arrive())
         par = {}
         for t in range(T):
-            st = t % S
-            prev = need[t - S] if t >= S else 0
-            for kind, stage, landed in (('k', stage_k, landed_k), ('v', stage_v, landed_v)):
-                for w in range(2):
-                    if (prev >> w) & 1:
-                        b = f'{kind}_empty{st}_{w}'
-                        p = par.get(b, 0)
-                        yield from wait(lambda b=b, p=p: bar(b).test(p))
-                        par[b] = p ^ 1
-                if any(op['reads'] == (kind, st) for op in pipe):
-                    raise Stale(f'{kind} stage {st} reloaded while an MMA reads it')
-                stage[st] = t
-                landed[st] = False
-                tma(kind, st, t)
+            for kind in (('k',) if split else ('k', 'v')):
+                yield from load(kind, t, par)
+
+    def producer_v():  # the V lane of the split producer
+        par = {}
+        for t in range(T):
+            yield from load('v', t, par)
 
     def issue(w, kind, t, j):
         st = t % S
@@ -193,7 +209,9 @@ def run(need, S, sep_p, seed, plant=None, max_steps=400000):
                 yield from pv(w)
 
         for t in range(T):
-            if plant != 'no_flush':
+            # single-loop producer: K(t) waits behind V(t - 1), which needs every
+            # PV of tile t - 1 - S
+            if not split and plant != 'no_flush':
                 yield from flush_below(t - S)
             yield from wait(lambda t=t: bar(f'k_full{t % S}').test((t // S) & 1))
             for w in range(2):
@@ -202,6 +220,11 @@ def run(need, S, sep_p, seed, plant=None, max_steps=400000):
                         yield from wait(lambda w=w: bar(f'q_full{w}').test(0))
                         q[w] = True
                     if pt[w] >= 0:
+                        # split producer: V(u) reuses the stage of tile u - S, so the
+                        # other warpgroup's PV of a tile <= u - S goes first
+                        o = 1 - w
+                        if split and plant != 'no_v_order' and 0 <= pt[o] <= pt[w] - S:
+                            yield from pv(o)
                         yield from pv(w)
                     issue(w, 'qk', t, c[w])
             for w in range(2):
@@ -229,6 +252,8 @@ def run(need, S, sep_p, seed, plant=None, max_steps=400000):
 
     live = {'producer': producer(), 'issuer': issuer_poll() if sep_p else issuer_fixed(),
             'wg0': softmax(0), 'wg1': softmax(1)}
+    if split:
+        live['producer_v'] = producer_v()
     idle = {k: 0 for k in live}
     for _ in range(max_steps):
         if not live and not events and not pipe:
@@ -347,13 +372,36 @@ def test_protocol_on_random_schedules(sep_p, S):
             assert run(need, S, sep_p, 100 * k + seed) == 'ok', need
 
 
-def test_planted_missing_flush_deadlocks():
-    # warpgroup 0 waits for K of a far tile while its own PV of an old tile,
-    # which the producer needs released first, is still unissued
+def test_planted_missing_flush_deadlocks_the_single_loop_producer():
+    # a producer that loads K(t) only after V(t - 1): warpgroup 0 waits for K of
+    # a far tile while its own PV of an old tile, which the producer needs
+    # released first, is still unissued
     need = [3, 2, 2, 2, 2, 2, 3]
-    results = {run(need, 2, False, seed, plant='no_flush') for seed in range(30)}
+    results = {run(need, 2, False, seed, plant='no_flush', split=False) for seed in range(30)}
     assert 'deadlock' in results
-    assert all(run(need, 2, False, seed) == 'ok' for seed in range(30))
+    assert all(run(need, 2, False, seed, split=False) == 'ok' for seed in range(30))
+
+
+def test_planted_missing_v_order_deadlocks_the_split_producer():
+    # split producer: warpgroup 1's PV of tile 0 is pending while warpgroup 0
+    # waits for V(2), which reuses tile 0's stage
+    need = [3, 1, 1, 1, 2]
+    results = {run(need, 2, False, seed, plant='no_v_order') for seed in range(60)}
+    assert 'deadlock' in results
+    assert all(run(need, 2, False, seed) == 'ok' for seed in range(60))
+
+
+@pytest.mark.parametrize("S", [2, 4])
+def test_split_producer_on_one_group_runs(S):
+    # long runs of tiles only one warpgroup needs, alternating: the case the
+    # split producer is for
+    for k in range(6):
+        rng = random.Random(k)
+        need = []
+        while len(need) < 40:
+            need += [rng.choice([1, 2])] * rng.randint(1, 6) + [3] * rng.randint(0, 2)
+        for seed in range(8):
+            assert run(need, S, False, 10 * k + seed) == 'ok', need
 
 
 def test_planted_unordered_k_test_reads_stale_data():

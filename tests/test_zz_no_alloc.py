@@ -17,7 +17,7 @@ import torch
 
 import workloads as W
 from oracle import select as OS
-from parity_util import bsa, f64, list_to_classes, selection_matches
+from parity_util import bsa, check_full_score_rows, f64, list_to_classes, selection_matches
 
 pytestmark = pytest.mark.gpu
 
@@ -81,6 +81,49 @@ def test_static_full_score_selection_matches_workspace_version_twice():
                 for row in (got[0, h, I], ref[0, h, I]):
                     ok, _ = selection_matches(row > 0, ap[I], groups, np.zeros(nb, bool))
                     assert ok, (h, I)
+
+
+def test_static_one_pass_in_two_chunks_equals_one_chunk():
+    """128 heads x 2048 tokens: the scratch holds the per-tile LSE slabs of 2032 of the 2048 query
+    blocks, so the static entry runs the one-pass form in two chunks; a caller workspace of the
+    reported size runs it in one. Every query block takes the same arithmetic either way: the
+    block lists are identical."""
+    m = bsa()
+    B, H, N, d, bs = 1, 128, 2048, 128, 128
+    q, k, _ = W.qkv_normal(B, H, N, d, 43)
+    nb = N // bs
+    dm = m.dims(B, H, N, d, bs, bs, 0)
+    spec = m.select_spec(m.SELECT_FULL_SCORE, [(0, nb - 2, 5), (nb - 2, nb, 1)], False, d ** -0.5)
+    qd, kd = q.cuda(), k.cuda()
+    ref = _with_workspace(m, dm, qd, kd, spec, nb, nb)
+    got = _static_via_c_abi(m, dm, qd, kd, spec, nb, nb)
+    for name in ("cnt", "idx", "flag", "bitmap"):
+        assert torch.equal(getattr(got, name), getattr(ref, name)), name
+
+
+def test_static_two_pass_form_agrees_with_the_one_pass_form():
+    """8 heads x 16384 tokens: too many slabs for the scratch's minimum chunk, so the static entry
+    runs the two-pass form (row LSE, then block sums with atomics) while the caller workspace runs
+    the one-pass form. Rows where the two differ must both be valid selections of the oracle's
+    A' (near-ties only), and they must be rare."""
+    m = bsa()
+    B, H, N, d, bs = 1, 8, 16384, 128, 128
+    q, k, _ = W.qkv_normal(B, H, N, d, 47)
+    nb = N // bs
+    groups = [(0, nb - 8, 38), (nb - 8, nb, 2)]
+    bias, _ = W.dlm_bias(H, nb, nb - 8, seed=11, n_col_pre=6, n_col_gen=1, windows=(2, 4))
+    dm = m.dims(B, H, N, d, bs, bs, 0)
+    spec = m.select_spec(m.SELECT_FULL_SCORE, groups, False, d ** -0.5)
+    qd, kd, bd = q.cuda(), k.cuda(), bias.cuda()
+    ref = list_to_classes(_with_workspace(m, dm, qd, kd, spec, nb, nb, bd), nb)
+    got = list_to_classes(_static_via_c_abi(m, dm, qd, kd, spec, nb, nb, bd), nb)
+    diff = [(h, I) for h in range(H) for I in range(nb) if not np.array_equal(got[0, h, I], ref[0, h, I])]
+    assert len(diff) <= H * nb // 50, len(diff)
+    for h in sorted({h for h, _ in diff}):
+        rows = np.array([I for hh, I in diff if hh == h])
+        for cls in (got, ref):
+            check_full_score_rows(cls[0, h], f64(q[0, h]), f64(k[0, h]), d ** -0.5, bs, bs, groups, rows,
+                                  bias=bias[h].numpy())
 
 
 def test_static_rejects_requests_beyond_its_scratch():
