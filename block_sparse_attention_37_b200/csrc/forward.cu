@@ -226,6 +226,9 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
           s | (int)(gb << kGrpShift) | (((pw >> lane) & 1u) ? kPart4 : 0);
     base += __popc(bal);
   }
+  // Each entry was written by the lane that kept it; the caller's lanes read
+  // entries other lanes wrote (tile reorder, geometry, tile counts).
+  __syncwarp();
   return base;
 }
 

@@ -28,6 +28,9 @@ __global__ void __launch_bounds__(256) block_pool_kernel(PoolParams p) {
   __shared__ float red[RPI][D + 1];
   __shared__ __align__(8) uint64_t full;
   __shared__ int no_abort;
+  // the selection kernel after this one may be scheduled now (it waits for
+  // this grid's completion before reading the pooled vectors)
+  asm volatile("griddepcontrol.launch_dependents;");
   const int I = blockIdx.x, bh = blockIdx.y, which = blockIdx.z;
   const int bs = which ? p.block_k : p.block_q;
   const int nb = which ? p.nKB : p.nQB;
@@ -102,6 +105,7 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 // One CTA per (b, h, query block). Block 256 threads.
 template <int D>
 __global__ void __launch_bounds__(256) select_kernel(SelectParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's output is complete
   extern __shared__ float sc[];  // [nKB] scores
   __shared__ int warp_tot[8];
   uint8_t* keep = reinterpret_cast<uint8_t*>(sc + p.nKB);
@@ -269,6 +273,7 @@ __device__ __forceinline__ void radix_cut(const float* sc, uint8_t* keep, int b,
 
 template <int D>
 __global__ void __launch_bounds__(256) select_rows_kernel(SelectParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the previous kernel's output is complete
   extern __shared__ float rsc[];  // [kRowsPerCta][nKB] scores, then [kRowsPerCta][nKB] keep bytes
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int per_bh = (p.nQB + kRowsPerCta - 1) / kRowsPerCta;
@@ -389,23 +394,36 @@ cudaError_t launch_block_pool(int d, const PoolParams& p, cudaStream_t stream) {
   return d == 64 ? launch_block_pool_d<64>(p, stream) : launch_block_pool_d<128>(p, stream);
 }
 
+// A programmatic dependent launch: the selection grid may be scheduled while
+// the kernel before it (pooling or the score pass) finishes; its kernels
+// wait on griddepcontrol.wait before reading anything that kernel wrote.
+template <class K>
+static cudaError_t launch_dependent(K kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t stream,
+                                   const SelectParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 cudaError_t launch_select(int d, const SelectParams& p, cudaStream_t stream) {
   if (p.nKB <= kRowsMaxKB) {
     const size_t smem = (size_t)kRowsPerCta * p.nKB * (sizeof(float) + 1);
     const unsigned grid = (unsigned)((size_t)p.B * p.H * ((p.nQB + kRowsPerCta - 1) / kRowsPerCta));
-    if (d == 64)
-      select_rows_kernel<64><<<grid, 32 * kRowsPerCta, smem, stream>>>(p);
-    else
-      select_rows_kernel<128><<<grid, 32 * kRowsPerCta, smem, stream>>>(p);
-    return cudaGetLastError();
+    return d == 64 ? launch_dependent(select_rows_kernel<64>, grid, 32 * kRowsPerCta, smem, stream, p)
+                   : launch_dependent(select_rows_kernel<128>, grid, 32 * kRowsPerCta, smem, stream, p);
   }
   const size_t smem = (size_t)p.nKB * sizeof(float) + (size_t)p.nKB;
   const unsigned grid = (unsigned)((size_t)p.B * p.H * p.nQB);
-  if (d == 64)
-    select_kernel<64><<<grid, 256, smem, stream>>>(p);
-  else
-    select_kernel<128><<<grid, 256, smem, stream>>>(p);
-  return cudaGetLastError();
+  return d == 64 ? launch_dependent(select_kernel<64>, grid, 256, smem, stream, p)
+                 : launch_dependent(select_kernel<128>, grid, 256, smem, stream, p);
 }
 
 }  // namespace bsa
