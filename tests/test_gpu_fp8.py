@@ -104,6 +104,34 @@ def _check_rows(got, q, k, v, mode, fn, rows, bias_fn=None, what="", mean_bar=5e
         assert err.mean() <= mean_bar, f"{what}: mean {float(err.mean()):.3e}"
 
 
+def test_forward_fp8_schedule_after_other_kernels():
+    """The forward's schedule is written lane by lane and read across lanes before the CTA's
+    barrier (e4m3 tile reorder, geometry, tile counts). Without a warp sync between the two,
+    the reorder could read what an earlier kernel left in shared memory. It then scrambled
+    the schedule: a misaligned-tile error, and at times an out-of-range scale index. Ragged
+    and even lengths in turn, each on fresh buffers after the other's kernels, many times;
+    every forward must end with the error word clear."""
+    m = bsa()
+    cases = []
+    for N in (128 * 6, 128 * 6 + 40):
+        w = W.arrow_case(B=1, H=4, n_text=128, grid_hw=(1, N - 128), d=128, block=128, seed=N,
+                         fracs=(0.25, 0.5, 0.25))
+        cases.append(w)
+    for rep in range(6):
+        for w in cases:
+            shp = w["shape"]
+            dm = _dims(shp)
+            ops = _quantize(dm, w["q"], w["k"], w["v"])
+            modes = torch.from_numpy(w["head_mode"]).cuda()
+            blocks = m.BlockList.empty(1, shp.H, shp.n_qb, shp.n_kb, bitmap=False)
+            m.build_mask(dm, m.MASK_ARROW, blocks, head_mode=modes, window=torch.from_numpy(w["window"]).cuda())
+            o = torch.empty(w["q"].shape, dtype=torch.bfloat16, device="cuda")
+            m.forward_fp8(dm, ops, o, modes, blocks=blocks, cache_in=w["cache"].cuda())
+            torch.cuda.synchronize()
+            assert m.get_device_error() == 0, (rep, shp.N)
+            del ops, blocks, o
+
+
 @pytest.mark.parametrize("N", [128 * 6, 128 * 6 + 40])
 def test_forward_fp8_arrow_full_skip(N):
     m = bsa()
