@@ -135,6 +135,20 @@ def test_workspace_sizes():
     assert bsa.select_workspace_size(dm2, sp2) >= 32 * 32768 * 4 + 32 * 256 * 256 * 4
 
 
+def test_full_score_workspace_below_the_reported_size_is_refused():
+    """bsa_select_topk's contract: at least bsa_select_workspace_size bytes. One 256-byte step
+    less is refused before any CUDA call, although the two-pass form would fit in it."""
+    bsa, lib = _lib()
+    dm = bsa.dims(1, 32, 32768, 128, 128, 128, 0)
+    sp = bsa.select_spec(bsa.SELECT_FULL_SCORE, [(0, 240, 72), (240, 256, 5)], False, 0.088)
+    need = bsa.select_workspace_size(dm, sp)
+    assert need > 32 * 32768 * 4 + 32 * 256 * 256 * 4  # the one-pass slabs are included
+    p = ctypes.c_void_p(256)
+    lst = bsa.BlockListC(p, p, p, None, 256)
+    assert lib.bsa_select_topk(ctypes.byref(dm), p, p, ctypes.byref(sp), None, p, need - 256,
+                               ctypes.byref(lst), None) == bsa.ERR_WORKSPACE
+
+
 def test_cpu_tensors_are_rejected():
     bsa, lib = _lib()
     import torch
