@@ -242,6 +242,19 @@ class ArrowJob(Job):
         if ev_fwd:
             ev_fwd[1].record()
 
+    def phases(self):
+        """The HBM-bound steps beside the forward: the plan search's RSE of this step's output
+        against the uncompressed output of the same inputs (every head FULL, computed once
+        here), each read once."""
+        bsa, s = self.bsa, self.s
+        if not hasattr(self, "o_full"):
+            self.o_full = torch.empty_like(self.q)
+            full = torch.zeros_like(self.modes)
+            bsa.forward(self.dm, self.q, self.k, self.v, self.o_full, full)
+            self.rse_out = torch.empty(4 * s.H, dtype=torch.float64, device="cuda")
+            torch.cuda.synchronize()
+        return [("rse", lambda: bsa.rse(self.dm, self.o, self.o_full, self.rse_out), rse_bytes(s.B, s.H, s.N, s.d))]
+
     def e2e_inputs(self):
         # Q, K, V, the mode table, the windows and (skip heads) the cached fp32 output
         return [t for t in (self.q, self.k, self.v, self.modes, self.wins, self.cache) if t is not None]
@@ -525,6 +538,11 @@ def job_throughput(flops_per_step: float, world: int, ms_per_step: float) -> flo
 
 def select_bytes(B, H, N, d):
     """Pooled selection: Q and K (bf16) read once; the pooled means and scores stay in L2."""
+    return 2 * B * H * N * d * 2
+
+
+def rse_bytes(B, H, N, d):
+    """The plan search's relative squared error: y_m and y_o (bf16) read once."""
     return 2 * B * H * N * d * 2
 
 

@@ -10,32 +10,47 @@
 
 namespace bsa {
 
-// Per head h (blockIdx.y): sum (y_m - y_o)^2, sum y_o and sum y_o^2 over
-// every batch item, token and channel, in fp64. Each thread reads 16-byte
-// chunks (8 bf16) of both tensors, grid-striding over the head's B * N * d
-// elements; a block reduces with warp shuffles and adds its three partial
-// sums to sums[3h .. 3h + 2] atomically.
-__global__ void __launch_bounds__(256) rse_kernel(const uint4* __restrict__ ym, const uint4* __restrict__ yo,
-                                                  int B, int H, long long chunks_per_bh, double* sums) {
-  const int h = blockIdx.y;
-  double num = 0.0, s = 0.0, ss = 0.0;
-  const long long per_head = (long long)B * chunks_per_bh;
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < per_head;
-       i += (long long)gridDim.x * blockDim.x) {
-    const long long b = i / chunks_per_bh;
-    const long long at = (b * H + h) * chunks_per_bh + (i - b * chunks_per_bh);
-    const uint4 a = __ldg(ym + at), o = __ldg(yo + at);
-    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, ow[4] = {o.x, o.y, o.z, o.w};
+// bf16 pairs of one 16-byte chunk of each tensor into the three fp64 sums.
+// bf16 -> fp32 is exact (the bf16 bits are the high half of the fp32), and so
+// is fp32 -> fp64.
+__device__ __forceinline__ void rse_add(const uint4& a, const uint4& o, double& num, double& s, double& ss) {
+  const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, ow[4] = {o.x, o.y, o.z, o.w};
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32
-      const double a0 = (double)__uint_as_float(aw[k] << 16), a1 = (double)__uint_as_float(aw[k] & 0xffff0000u);
-      const double o0 = (double)__uint_as_float(ow[k] << 16), o1 = (double)__uint_as_float(ow[k] & 0xffff0000u);
-      num += (a0 - o0) * (a0 - o0) + (a1 - o1) * (a1 - o1);
-      s += o0 + o1;
-      ss += o0 * o0 + o1 * o1;
-    }
+  for (int k = 0; k < 4; ++k) {
+    const double a0 = (double)__uint_as_float(aw[k] << 16), a1 = (double)__uint_as_float(aw[k] & 0xffff0000u);
+    const double o0 = (double)__uint_as_float(ow[k] << 16), o1 = (double)__uint_as_float(ow[k] & 0xffff0000u);
+    num += (a0 - o0) * (a0 - o0) + (a1 - o1) * (a1 - o1);
+    s += o0 + o1;
+    ss += o0 * o0 + o1 * o1;
   }
+}
+
+// Per head h (blockIdx.y) and batch item b (blockIdx.z): sum (y_m - y_o)^2,
+// sum y_o and sum y_o^2 over the item's tokens and channels, in fp64. The
+// (b, h) slab is one contiguous run of 16-byte chunks (8 bf16); the blocks of
+// the slab grid-stride over it with four chunk pairs in flight per thread. A
+// block reduces with warp shuffles and adds its three partial sums to
+// sums[3h .. 3h + 2] atomically.
+__global__ void __launch_bounds__(256) rse_kernel(const uint4* __restrict__ ym, const uint4* __restrict__ yo,
+                                                  int H, long long chunks_per_bh, double* sums) {
+  const int h = blockIdx.y;
+  const long long base = ((long long)blockIdx.z * H + h) * chunks_per_bh;
+  const uint4* pa = ym + base;
+  const uint4* po = yo + base;
+  double num = 0.0, s = 0.0, ss = 0.0;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < chunks_per_bh; i += 4 * stride) {
+    uint4 a[4], o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      a[u] = __ldg(pa + i + u * stride);
+      o[u] = __ldg(po + i + u * stride);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) rse_add(a[u], o[u], num, s, ss);
+  }
+  for (; i < chunks_per_bh; i += stride) rse_add(__ldg(pa + i), __ldg(po + i), num, s, ss);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) {
     num += __shfl_down_sync(0xffffffffu, num, off);
@@ -79,15 +94,16 @@ extern "C" int bsa_rse(const bsa_dims* dims, const void* y_m, const void* y_o, d
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   double* sums = out + dims->H;
   if (cudaMemsetAsync(sums, 0, sizeof(double) * 3 * (size_t)dims->H, st) != cudaSuccess) return BSA_ERR_CUDA;
-  // enough blocks per head to cover the SMs a few times over
-  const long long per_head = (long long)dims->B * (nd / 8);
-  long long bx = (4ll * num_sms() + dims->H - 1) / dims->H;
-  const long long need = (per_head + 255) / 256;
+  // one grid slab per (b, h), with enough blocks per slab to give every SM
+  // about eight blocks
+  if (dims->B > 65535 || dims->H > 65535) return BSA_ERR_UNSUPPORTED;
+  const long long slabs = (long long)dims->B * dims->H;
+  long long bx = (8ll * num_sms() + slabs - 1) / slabs;
+  const long long need = (nd / 8 + 255) / 256;
   if (bx > need) bx = need;
   if (bx < 1) bx = 1;
-  rse_kernel<<<dim3((unsigned)bx, (unsigned)dims->H), 256, 0, st>>>(static_cast<const uint4*>(y_m),
-                                                                    static_cast<const uint4*>(y_o), dims->B,
-                                                                    dims->H, nd / 8, sums);
+  rse_kernel<<<dim3((unsigned)bx, (unsigned)dims->H, (unsigned)dims->B), 256, 0, st>>>(
+      static_cast<const uint4*>(y_m), static_cast<const uint4*>(y_o), dims->H, nd / 8, sums);
   if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   rse_finalize<<<1, 256, 0, st>>>(sums, out, dims->H, (double)dims->B * (double)nd);
   return cuda_status(cudaGetLastError());

@@ -293,7 +293,7 @@ int bsa_unpermute_tiles(const bsa_dims* dims, const bsa_gna_geom* geom, int32_t 
  *    out[H + 3h + 0..2] = sum (y_m - y_o)^2, sum y_o, sum y_o^2 (fp64).
  *    A head whose y_o is constant has a zero denominator (I = inf or NaN).
  *  Errors: INVALID_ARG (null pointer, bad dims), UNSUPPORTED (N*d not a
- *  multiple of 8), CUDA. */
+ *  multiple of 8, or B or H above 65535), CUDA. */
 int bsa_rse(const bsa_dims* dims, const void* y_m, const void* y_o, double* out, void* stream);
 
 /* bsa_plan_heads: the head-wise compression plan of one layer and step
