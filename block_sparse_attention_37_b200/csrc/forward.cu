@@ -6,10 +6,11 @@
 // 128-key tile none of its rows keeps, so each tile costs tensor work only
 // for the warpgroups that need it while K and V are loaded once.
 // Roles (384 threads, three aligned warpgroups):
-//   warp 0      TMA producer: both Q tiles, then K/V tiles into a shared ring
+//   warp 0      TMA producer: both Q tiles, then the K tiles into their ring
 //   warp 1      TMEM allocator and tcgen05.mma issuer (whole warp, one
 //               elected lane issues)
-//   warps 2-3   idle (they complete the control warpgroup)
+//   warp 2      TMA producer of the V tiles into their own ring
+//   warp 3      idle (it completes the control warpgroup)
 //   warps 4-7   softmax warpgroup 0 (rows 0..127 of the CTA)
 //   warps 8-11  softmax warpgroup 1 (rows 128..255)
 // The control warpgroup hands registers to the softmax warpgroups
@@ -84,6 +85,22 @@ static_assert(FwdCfg<64, false>::SMEM_ALLOC <= 227 * 1024 && FwdCfg<128, false>:
 constexpr int kGrpShift = 24;
 constexpr int kPart4 = 1 << 28;
 
+// Mask kind a kernel is compiled for. kMaskAny reads it from the parameters
+// (no mask, GNA in any layout); kMaskGnaSlice is GNA in a layout whose 64-key
+// segments each lie in one slice of a tile, the form whose fine mask comes
+// from the precomputed segment geometry. Compiling that form alone leaves the
+// general GNA decoder out of its code.
+constexpr int kMaskAny = 0;
+constexpr int kMaskGnaSlice = 1;
+template <int MK>
+__device__ __forceinline__ bool gna_on(const AttnParams& p) {
+  return MK == kMaskGnaSlice || p.has_gna;
+}
+template <int MK>
+__device__ __forceinline__ bool gna_slice(const AttnParams& p) {
+  return MK == kMaskGnaSlice || (p.has_gna && p.g.seg_one_slice);
+}
+
 template <int N>
 __device__ __forceinline__ void regs_release() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
@@ -116,6 +133,7 @@ __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.w
 // window loses that group's bit (the group needs neither its QK^T nor its
 // PV), and a segment no group needs is left out. `pairs`: segments are kept
 // or left out in aligned pairs (the e4m3 V loads take 128-key runs).
+template <int MK>
 __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0, uint32_t* vb,
                                  uint32_t* pb, int32_t* sched, int lane, bool pairs) {
   const int nwords = (p.nSeg + 31) >> 5;
@@ -124,7 +142,7 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
   const int spb = p.block_k >> 6;
   if (mode == BSA_HEAD_FULL) {
     for (int w = lane; w < nwords; w += 32) vb[w] = bit_range(0, min(32, p.nSeg - w * 32));
-    if (p.has_gna && p.g.has_padding)
+    if (gna_on<MK>(p) && p.g.has_padding)
       for (int J = lane; J < p.nKB; J += 32) {
         if (!gna_block_padded(p.g, J)) continue;
         for (int u = 0; u < spb; ++u) {
@@ -166,7 +184,7 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
           continue;
         }
         bool part = p.flag[at] == BSA_BLOCK_PARTIAL;
-        if (part && !p.has_gna) {
+        if (part && !gna_on<MK>(p)) {
           record_error(BSA_DEVERR_NO_GEOMETRY);
           part = false;
         }
@@ -189,7 +207,7 @@ __device__ int build_schedule256(const AttnParams& p, int mode, int bh, int row0
   }
   __syncwarp();
   // the groups' windows (lane g computes group g's, then every lane gets all four)
-  const bool narrow = mode != BSA_HEAD_FULL && p.has_gna && p.g.seg_one_slice;
+  const bool narrow = mode != BSA_HEAD_FULL && gna_slice<MK>(p);
   GroupWin gw[4];
   if (narrow) {
     GroupWin mine{0, 0, 0, 0, 0, 0, false};
@@ -435,7 +453,7 @@ __device__ void skip_copy256(const AttnParams& p, int bh, int row0) {
   }
 }
 
-template <int D, bool F8 = false>
+template <int D, bool F8 = false, int MK = kMaskAny>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -519,12 +537,12 @@ __global__ void __launch_bounds__(384, 1)
     tmem_relinquish();
   }
   if (warp == 0) {
-    const int n = build_schedule256(p, mode, bh, row0, vb, vb + 256, sched, lane, F8);
+    const int n = build_schedule256<MK>(p, mode, bh, row0, vb, vb + 256, sched, lane, F8);
     // tiles each warpgroup needs
     const int act = 1 | ((row0 + 128 < p.N) ? 2 : 0);
     if constexpr (F8) reorder_tiles(sched, reinterpret_cast<int32_t*>(smem + C::TMP_OFF), n, act, lane);
     // where every partial segment sits in the grid, once for the whole CTA
-    if (p.has_gna && p.g.seg_one_slice) {
+    if (gna_slice<MK>(p)) {
       uint64_t* geo = reinterpret_cast<uint64_t*>(smem + C::GEO_OFF);
       for (int i = lane; i < n; i += 32) {
         const int e = sched[i];
@@ -894,9 +912,9 @@ __global__ void __launch_bounds__(384, 1)
     const size_t bias_row = ((size_t)h * p.nQB + Iq) * p.nKB;
     const int my_bit = 1 << (kGrpShift + grp);
 
-    const QWin qw = gna_query_window(p.g, pq, p.has_gna && mode == BSA_HEAD_SPARSE);
+    const QWin qw = gna_query_window(p.g, pq, gna_on<MK>(p) && mode == BSA_HEAD_SPARSE);
     const QBox qb = gna_query_box(p.g, qw);
-    const bool geo_fast = p.has_gna && p.g.seg_one_slice;
+    const bool geo_fast = gna_slice<MK>(p);
     const uint64_t* geo = reinterpret_cast<const uint64_t*>(smem + C::GEO_OFF);
 
     const float cscale = p.scale_log2;
@@ -932,12 +950,12 @@ __global__ void __launch_bounds__(384, 1)
         mb = 0ull;
         if (ea & my_bit) {
           ma = tail_bits(p.N, sa);
-          if ((ea & kPart4) && p.has_gna)
+          if ((ea & kPart4) && gna_on<MK>(p))
             ma &= geo_fast ? gna_segment_bits_geo(p.g, sa, geo[2 * t], qb) : gna_segment_bits(p.g, sa, qw);
         }
         if (eb >= 0 && (eb & my_bit)) {
           mb = tail_bits(p.N, sb);
-          if ((eb & kPart4) && p.has_gna)
+          if ((eb & kPart4) && gna_on<MK>(p))
             mb &= geo_fast ? gna_segment_bits_geo(p.g, sb, geo[2 * t + 1], qb) : gna_segment_bits(p.g, sb, qw);
         }
       }
@@ -1146,11 +1164,11 @@ __global__ void __launch_bounds__(384, 1)
   }
 }
 
-template <int D, bool F8>
+template <int D, bool F8, int MK = kMaskAny>
 static cudaError_t launch_fwd_d(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                 const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
   using C = FwdCfg<D, F8>;
-  auto fn = fwd_kernel<D, F8>;
+  auto fn = fwd_kernel<D, F8, MK>;
   static DeviceOnce once;
   const cudaError_t e = once.run([&]() -> cudaError_t {
     // the register split needs the full launch allocation: a smaller one
@@ -1169,6 +1187,7 @@ static cudaError_t launch_fwd_d(const CUtensorMap& q, const CUtensorMap& k, cons
 cudaError_t launch_forward(int d, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                            const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
   if (d == 64) return launch_fwd_d<64, false>(q, k, v, o, p, grid, stream);
+  if (p.has_gna && p.g.seg_one_slice) return launch_fwd_d<128, false, kMaskGnaSlice>(q, k, v, o, p, grid, stream);
   return launch_fwd_d<128, false>(q, k, v, o, p, grid, stream);
 }
 
