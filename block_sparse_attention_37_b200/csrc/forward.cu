@@ -1193,6 +1193,7 @@ cudaError_t launch_forward(int d, const CUtensorMap& q, const CUtensorMap& k, co
 
 cudaError_t launch_forward_fp8(const CUtensorMap& q8, const CUtensorMap& k8, const CUtensorMap& v8t,
                                const CUtensorMap& o, const AttnParams& p, int grid, cudaStream_t stream) {
+  if (p.has_gna && p.g.seg_one_slice) return launch_fwd_d<128, true, kMaskGnaSlice>(q8, k8, v8t, o, p, grid, stream);
   return launch_fwd_d<128, true>(q8, k8, v8t, o, p, grid, stream);
 }
 
