@@ -227,6 +227,11 @@ def _gna_forward(B, H, n_text, grid, tile, window, stride, d, seed, modes, rows_
     (50, (5, 9, 20), (2, 4, 8), (3, 5, 7), (1, 2, 2)),      # padding in grid and text
     (0, (300,), (64,), (97,), (5,)),                          # 1-D, padded last tile
     (128, (8, 256), (1, 128), (3, 48), (1, 16)),              # x tile wider than a segment
+    # one-slice layouts (each 64-key segment in one y-x slice of a tile), with padding: the
+    # forward's instantiation for them, and the per-group narrowing of partial segments
+    (128, (4, 12, 20), (2, 8, 8), (3, 9, 11), (1, 1, 1)),
+    (128, (4, 12, 20), (2, 8, 8), (3, 9, 11), (1, 3, 2)),
+    (40, (3, 20, 10), (1, 16, 4), (3, 7, 5), (1, 2, 1)),      # block 64, padded text
 ])
 def test_forward_gna_small(n_text, grid, tile, window, stride):
     _gna_forward(1, 3, n_text, grid, tile, window, stride, 128, 7, modes=[1, 0, 1])

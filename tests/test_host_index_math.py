@@ -137,6 +137,9 @@ CASES = [
     (256, (16, 48, 80), (4, 8, 8), (8, 16, 24), (4, 8, 8)),     # the video workload, stride 4x8x8
     (33, (3, 37, 21), (1, 16, 8), (2, 9, 11), (1, 2, 3)),       # segments in one t-slice, two per slice
     (0, (40, 50), (8, 8), (7, 9), (1, 1)),                      # 2-D, one segment per tile, padded y
+    (128, (4, 12, 20), (2, 8, 8), (3, 9, 11), (1, 1, 1)),       # one-slice, padded y and x
+    (128, (4, 12, 20), (2, 8, 8), (3, 9, 11), (1, 3, 2)),       # the same, strided
+    (40, (3, 20, 10), (1, 16, 4), (3, 7, 5), (1, 2, 1)),        # one-slice, block 64, padded text
 ]
 
 
